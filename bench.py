@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Throughput of chunked KDA prefill on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 5]
+
+A step is one kda_forward over the large prefill (B=4, Nqk=Nv=32, S=16384, D=128, BNSD; seeded
+synthetic bf16 inputs ~ N(0,1)).  Units (sequence, value head) are independent, so N > 1 runs one
+replica of the workload per GPU with no collective on the data path (weak scaling); torchrun
+supplies RANK / LOCAL_RANK / WORLD_SIZE.  ``--impl reference`` times the fp64 CPU oracle on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_workloads as W  # noqa: E402
+
+METRIC = "KDA prefill tokens/s per B200 (B·Nv·S/s) and % of tensor/HBM roofline"
+UNIT = "token-heads/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML)
+# ----------------------------------------------------------------------------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period, self.ok = period_s, False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clocks rather than guess
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in _REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# roofline bookkeeping
+# ----------------------------------------------------------------------------
+
+def algorithmic_bytes(w: W.Workload, with_initial_state: bool) -> int:
+    """Unique HBM bytes of one forward: q,k (per qk head), v, g, beta, out, states, params."""
+    rows = w.S if w.layout == "TND" else w.B * w.S
+    qk = 2 * rows * w.Nqk * w.D * 2
+    vg_out = 3 * rows * w.Nv * w.D * 2
+    beta = rows * w.Nv * 2
+    states = (2 if with_initial_state else 1) * w.B * w.Nv * w.D * w.D * 4
+    params = w.Nv * 4 + w.Nv * w.D * 4
+    return qk + vg_out + beta + states + params
+
+
+def algorithmic_flops(w: W.Workload) -> float:
+    """Dense MMA flops of the chunked method per chunk-head (C=64, D=128): 11.62 MFLOP."""
+    per_chunk = 5 * 2 * 64 * 64 * 128 + 3 * 2 * 64 * 128 * 128
+    chunks = sum(math.ceil(L / 64) for L in w.lengths) * w.Nv
+    return float(per_chunk * chunks)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "chunked_kda_prefill_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernels."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("kernel_source_sha") == kernel_source_hash():
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ----------------------------------------------------------------------------
+
+def cpu_oracle_sample(w: W.Workload, inp: dict, budget_s: float = 10.0, tokens: int | None = None):
+    """Time the fp64 oracle (recurrence) on batches of whole units until ``budget_s`` elapses.
+
+    One batch is one unit per host thread.  ``tokens`` keeps only the first ``tokens`` rows of
+    every sequence (BNSD/BSND), a bounded sample with the same per-token work.
+    """
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    it, lengths, S = inp, list(w.lengths), w.S
+    if tokens is not None and w.layout != "TND" and tokens < w.S:
+        it = dict(inp)
+        for n in ("q", "k", "v", "g", "beta"):
+            it[n] = inp[n][:, :, :tokens] if w.layout == "BNSD" else inp[n][:, :tokens]
+        lengths, S = [min(L, tokens) for L in w.lengths], tokens
+    cu = np.concatenate([[0], np.cumsum(lengths)]) if w.layout != "TND" else w.cu_seqlens
+    units = [(b, h) for b in range(w.B) for h in range(w.Nv)]
+    oracle.lib()
+    done_tokens, n_units, i = 0, 0, 0
+    t0 = time.perf_counter()
+    while i < len(units):
+        batch = units[i:i + cores]
+        i += cores
+        oracle.run_units(it, w.layout, w.B, w.Nqk, w.Nv, S, w.D, w.scale, w.lower_bound, cu,
+                         units=batch, form="recurrent", threads=cores)
+        done_tokens += sum(lengths[b] for b, _ in batch)
+        n_units += len(batch)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_units} whole (sequence, value head) units of {w.name}"
+                      + ("" if tokens is None else f", first {tokens} tokens each")
+                      + f", fp64 recurrence, {dt:.1f} s wall on {cores} threads"}, dt
+
+
+# ----------------------------------------------------------------------------
+# runs
+# ----------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = W.workload(args.workload)
+    inp = W.generate(w)
+    cores = len(os.sched_getaffinity(0))
+    tokens = args.ref_tokens
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, inp, budget_s=0.0, tokens=min(tokens, 256))
+    times, tok = [], 0
+    for _ in range(args.steps):
+        r, dt = cpu_oracle_sample(w, inp, budget_s=0.0, tokens=tokens)
+        times.append(dt)
+        tok += r["value"] * dt
+    total = sum(times)
+    value = tok / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"each step: the first {tokens} tokens of {min(cores, w.units)}"
+                                       f" (sequence, value head) units of {w.name}, fp64 "
+                                       "recurrence, one unit per host thread"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w: W.Workload, world: int):
+    c = w.describe()
+    c["parallelism"] = ("single GPU" if world == 1 else
+                        f"{world} replicas, one independent copy of the workload per GPU")
+    rows = w.S if w.layout == "TND" else w.B * w.S
+    in_bytes = 5 * rows * w.Nv * w.D * 2
+    c["l2"] = (f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2 (126 MB); no flush"
+               if in_bytes > 126e6 else "L2 flushed between steps by a 256 MB write")
+    return c
+
+
+def run_ours(args, rank, world):
+    import torch
+    import chunked_kda_prefill_b200 as kda
+
+    local = _env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    w = W.workload(args.workload)
+    if world > 1:
+        w.seed = w.seed + 1000 * rank
+    inp = W.generate(w)
+    host = {}
+    for n in ("q", "k", "v", "g", "beta"):
+        host[n] = torch.from_numpy(np.ascontiguousarray(inp[n]).view(np.int16)).view(
+            torch.bfloat16).pin_memory()
+    for n in ("A_log", "dt_bias", "initial_state"):
+        host[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).pin_memory()
+    d = {n: t.to(dev) for n, t in host.items()}
+    cu = w.cu_seqlens if (w.layout == "TND" or any(L != w.S for L in w.lengths)) else None
+    plan = kda.plan(d["q"], d["v"], d["initial_state"], w.layout, cu_seqlens=cu)
+    ws = plan.workspace()
+    out = torch.empty_like(d["v"])
+    fs = torch.empty((w.B, w.Nv, w.D, w.D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    small_l2 = 5 * (w.S if w.layout == "TND" else w.B * w.S) * w.Nv * w.D * 2 <= 126e6
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if small_l2 else None
+
+    def fwd():
+        kda.flash_kda(d["q"], d["k"], d["v"], d["g"], d["beta"], w.scale, d["initial_state"],
+                      d["A_log"], d["dt_bias"], w.lower_bound, w.layout, plan, out=out,
+                      final_state=fs, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            if flush is not None:
+                flush.zero_()
+            fwd()
+    kda.device_status(ws, stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+
+    # ---- device-resident timed region ----
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fl_ms = 0.0
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(dev)
+        barrier()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(args.steps):
+                if flush is not None:
+                    flush.zero_()
+                fwd()
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    elapsed_ms = start.elapsed_time(end)
+    if flush is not None:  # time the flushes alone and take them out of the kernel time
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for _ in range(args.steps):
+                flush.zero_()
+            f1.record(stream)
+        torch.cuda.synchronize(dev)
+        fl_ms = f0.elapsed_time(f1)
+    kda.device_status(ws, stream)
+    elapsed_ms = _max_over_ranks(elapsed_ms, dist, dev)
+    kernel_ms = (elapsed_ms - fl_ms) / args.steps
+
+    # ---- end to end: pinned host inputs -> device -> forward -> host outputs ----
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        fs_h = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * 2 + fs_h.numel() * 4
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps_e2e = max(1, min(args.steps, args.e2e_steps))
+        torch.cuda.synchronize(dev)
+        barrier()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps_e2e):
+                for n, t in host.items():
+                    d[n].copy_(t, non_blocking=True)
+                fwd()
+                out_h.copy_(out, non_blocking=True)
+                fs_h.copy_(fs, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = _max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        e2e = {"value": world * w.token_heads * steps_e2e / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": steps_e2e}
+
+    value = world * w.token_heads * args.steps / (elapsed_ms / 1e3)
+    peak, peak_kind = measured_peaks()
+    abytes = algorithmic_bytes(w, True)
+    achieved = abytes / (kernel_ms / 1e3) / 1e9
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 inputs, random-init A_log/dt_bias)",
+            "config": _config(w, world), "clocks": clk.report(), "e2e": e2e,
+            "gpu_launches": args.steps * kda.kernels_per_forward(),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": ncu_traffic(w.name),
+                         "kernel": kda.forward_kernel_names(),
+                         "algorithmic_bytes": abytes, "kernel_ms": kernel_ms,
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "tensor_tflops": algorithmic_flops(w) / (kernel_ms / 1e3) / 1e12}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"], _ = cpu_oracle_sample(w, inp, budget_s=args.cpu_budget)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def _max_over_ranks(x, dist, dev):
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-tokens", type=int, default=4096)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,9 @@
+"""B200-native chunked Kimi Delta Attention (KDA) prefill.
+
+Hand-written sm_100a CUDA kernels behind a C ABI (include/kda.h, libkda.so); this package is
+the thin Python binding over it.  Build the library with
+``python -m chunked_kda_prefill_b200.build``.
+"""
+from ._lib import EXPORTS, LIB_PATH, KdaError, KdaShape, load  # noqa: F401
+from .api import (KdaPlan, LAYOUTS, device_status, flash_kda, forward_kernel_names,  # noqa: F401
+                  kernels_per_forward, make_plan, plan)

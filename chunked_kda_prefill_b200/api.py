@@ -1,0 +1,167 @@
+"""Python API over libkda.so, mirroring flash_kda_metadata / flash_kda (FlashKDA README, 快速开始).
+
+    plan = chunked_kda_prefill_b200.plan(q, v, initial_state, "BNSD", cu_seqlens=None)
+    out, final_state = chunked_kda_prefill_b200.flash_kda(
+        q, k, v, g, beta, 1 / math.sqrt(128), initial_state, A_log, dt_bias, -5.0, "BNSD", plan)
+
+PyTorch supplies device memory and the current stream; the functions below only pass
+pointers and sizes to the C ABI (include/kda.h).
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import KdaError, KdaShape, check
+
+LAYOUTS = {"BNSD": 0, "BSND": 1, "TND": 2}
+
+
+@dataclass
+class KdaPlan:
+    """Host + device copies of the int32 schedule, and the workspace size it needs."""
+    shape: KdaShape
+    layout: str
+    host: np.ndarray
+    dev: torch.Tensor
+    workspace_bytes: int
+    cu_seqlens: np.ndarray | None
+    _workspace: torch.Tensor | None = None
+
+    @property
+    def n_units(self) -> int:
+        return int(self.host[4])
+
+    @property
+    def total_chunks(self) -> int:
+        return int(self.host[11])
+
+    def workspace(self) -> torch.Tensor:
+        """A workspace owned by the plan, allocated on first use and reused afterwards."""
+        if self._workspace is None or self._workspace.device != self.dev.device:
+            self._workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8,
+                                          device=self.dev.device)
+        return self._workspace
+
+
+def _shape_from(q: torch.Tensor, v: torch.Tensor, layout: str, cu_seqlens) -> KdaShape:
+    if layout not in LAYOUTS:
+        raise KdaError(2, f"layout {layout!r}")
+    if layout == "BNSD":
+        B, Nqk, S, D = q.shape
+        Nv = v.shape[1]
+    elif layout == "BSND":
+        B, S, Nqk, D = q.shape
+        Nv = v.shape[2]
+    else:
+        if cu_seqlens is None:
+            raise KdaError(7, "TND layout needs cu_seqlens")
+        S, Nqk, D = q.shape
+        Nv = v.shape[1]
+        B = len(cu_seqlens) - 1
+    return KdaShape(LAYOUTS[layout], int(B), int(Nqk), int(Nv), int(S), int(D))
+
+
+def make_plan(shape: KdaShape, layout: str, cu_seqlens=None, num_sms: int | None = None,
+              device=None) -> KdaPlan:
+    """Build a plan from an explicit shape (host work only, plus one small device copy)."""
+    L = _lib.load()
+    n = ctypes.c_size_t(0)
+    check(L.kda_plan_size(ctypes.byref(shape), ctypes.byref(n)), "kda_plan_size")
+    host = np.zeros(n.value, dtype=np.int32)
+    cu = None
+    cu_ptr = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64)).astype(np.int32)
+        cu_ptr = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    if num_sms is None:
+        num_sms = (torch.cuda.get_device_properties(device).multi_processor_count
+                   if torch.cuda.is_available() else 148)
+    check(L.kda_plan(ctypes.byref(shape), cu_ptr, int(num_sms),
+                     host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), host.size), "kda_plan")
+    ws = ctypes.c_size_t(0)
+    check(L.kda_workspace_size(host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), host.size,
+                               ctypes.byref(ws)), "kda_workspace_size")
+    if device is not None and torch.cuda.is_available():
+        dev = torch.from_numpy(host).to(device)
+    else:
+        dev = torch.from_numpy(host.copy())
+    return KdaPlan(shape, layout, host, dev, int(ws.value), cu)
+
+
+def plan(q: torch.Tensor, v: torch.Tensor, initial_state: torch.Tensor | None, layout: str,
+         cu_seqlens=None, num_sms: int | None = None) -> KdaPlan:
+    """flash_kda_metadata counterpart: shapes, layout and valid lengths -> schedule."""
+    if isinstance(cu_seqlens, torch.Tensor):
+        cu_seqlens = cu_seqlens.detach().to("cpu").numpy()
+    shape = _shape_from(q, v, layout, cu_seqlens)
+    if initial_state is not None and initial_state.shape[0] != shape.B:
+        raise KdaError(3, "initial_state batch does not match the number of sequences")
+    return make_plan(shape, layout, cu_seqlens, num_sms, device=q.device)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _expect(t, name, dtype, device):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+
+
+def flash_kda(q, k, v, g, beta, scale: float, initial_state, A_log, dt_bias, lower_bound: float,
+              layout: str, plan: KdaPlan, out: torch.Tensor | None = None,
+              final_state: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """The fused forward pass. Returns (out, final_state); out has v's shape and layout."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("flash_kda runs on a CUDA device only")
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta")):
+        _expect(t, name, torch.bfloat16, dev)
+    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias")):
+        _expect(t, name, torch.float32, dev)
+    if initial_state is not None:
+        _expect(initial_state, "initial_state", torch.float32, dev)
+    if plan.layout != layout:
+        raise KdaError(8, "plan was built for another layout")
+    sh = plan.shape
+    if out is None:
+        out = torch.empty_like(v)
+    if final_state is None:
+        final_state = torch.empty((sh.B, sh.Nv, sh.D, sh.D), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = plan.workspace()
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    L = _lib.load()
+    code = L.kda_forward(ctypes.byref(sh), plan.host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                         plan.dev.data_ptr(), plan.host.size, q.data_ptr(), k.data_ptr(),
+                         v.data_ptr(), g.data_ptr(), beta.data_ptr(), float(scale),
+                         _ptr(initial_state), A_log.data_ptr(), dt_bias.data_ptr(),
+                         float(lower_bound), workspace.data_ptr(), workspace.numel(),
+                         out.data_ptr(), final_state.data_ptr(), s.cuda_stream)
+    check(code, "kda_forward")
+    return out, final_state
+
+
+def device_status(workspace: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+    """Synchronise and raise if the last forward on this workspace recorded a device error."""
+    s = stream if stream is not None else torch.cuda.current_stream(workspace.device)
+    check(_lib.load().kda_device_status(workspace.data_ptr(), s.cuda_stream), "kda_device_status")
+
+
+def kernels_per_forward() -> int:
+    """Kernels of this library that one kda_forward launches."""
+    return 2
+
+
+def forward_kernel_names() -> str:
+    return "kda_chunk_simt_kernel + kda_scan_simt_kernel"

@@ -1,0 +1,133 @@
+// kda_api.cu -- kda_forward / kda_device_status: argument checks, then the kernel launches.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "kda_internal.h"
+#include "kda_layout.cuh"
+
+namespace kda {
+namespace {
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+Range range_of(const void* p, size_t bytes) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return {lo, lo + bytes};
+}
+
+// Checks that the current device is an sm_100 part; cached per device ordinal.
+kda_status_t check_device() {
+  static int checked[64] = {0};  // 0 unknown, 1 ok, 2 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && checked[dev]) return checked[dev] == 1 ? KDA_OK : KDA_ERR_DEVICE;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  const bool ok = (major == 10);
+  if (dev >= 0 && dev < 64) checked[dev] = ok ? 1 : 2;
+  return ok ? KDA_OK : KDA_ERR_DEVICE;
+}
+
+}  // namespace
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* plan_host,
+                                    const int32_t* plan_dev, size_t n_int32, const void* q,
+                                    const void* k, const void* v, const void* g, const void* beta,
+                                    float scale, const float* initial_state, const float* A_log,
+                                    const float* dt_bias, float lower_bound, void* workspace,
+                                    size_t workspace_bytes, void* out, float* final_state,
+                                    kda_stream_t stream) {
+  kda_status_t st = validate_shape(shape);
+  if (st != KDA_OK) return st;
+  if (!plan_host || !plan_dev || !q || !k || !v || !g || !beta || !A_log || !dt_bias ||
+      !workspace || !out || !final_state)
+    return KDA_ERR_NULL;
+  st = validate_plan(plan_host, n_int32, shape);
+  if (st != KDA_OK) return st;
+  if (!std::isfinite(scale)) return KDA_ERR_LOWER_BOUND;
+  if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_LOWER_BOUND;
+
+  {
+    const void* a16[] = {q, k, v, g, out, final_state, A_log, dt_bias, plan_dev, initial_state};
+    for (const void* ptr : a16)
+      if (reinterpret_cast<uintptr_t>(ptr) & 15u) return KDA_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(beta) & 1u) return KDA_ERR_ALIGN;
+  }
+  size_t need = 0;
+  st = kda_workspace_size(plan_host, n_int32, &need);
+  if (st != KDA_OK) return st;
+  if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return KDA_ERR_WORKSPACE;
+
+  // aliasing: outputs must not overlap any input or each other
+  const long long rows =
+      shape->layout == KDA_LAYOUT_TND ? (long long)shape->S : (long long)shape->B * shape->S;
+  const size_t qk_bytes = (size_t)rows * shape->Nqk * kD * 2;
+  const size_t vg_bytes = (size_t)rows * shape->Nv * kD * 2;
+  const size_t beta_bytes = (size_t)rows * shape->Nv * 2;
+  const size_t st_bytes = (size_t)shape->B * shape->Nv * kD * kD * 4;
+  const Range r_out = range_of(out, vg_bytes), r_fs = range_of(final_state, st_bytes);
+  const Range ins[] = {range_of(q, qk_bytes), range_of(k, qk_bytes), range_of(v, vg_bytes),
+                       range_of(g, vg_bytes), range_of(beta, beta_bytes),
+                       range_of(workspace, need), range_of(plan_dev, n_int32 * 4),
+                       initial_state ? range_of(initial_state, st_bytes) : Range{0, 0}};
+  for (const Range& r : ins) {
+    if (r.hi == 0) continue;
+    if (overlaps(r, r_out) || overlaps(r, r_fs)) return KDA_ERR_ALIAS;
+  }
+  if (overlaps(r_out, r_fs)) return KDA_ERR_ALIAS;
+
+  st = check_device();
+  if (st != KDA_OK) return st;
+
+  Params p{};
+  p.layout = shape->layout;
+  p.B = shape->B;
+  p.Nqk = shape->Nqk;
+  p.Nv = shape->Nv;
+  p.S = shape->S;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.g = static_cast<const __nv_bfloat16*>(g);
+  p.beta = static_cast<const __nv_bfloat16*>(beta);
+  p.scale = scale;
+  p.S0 = initial_state;
+  p.A_log = A_log;
+  p.dt_bias = dt_bias;
+  p.lower_bound = lower_bound;
+  p.plan = plan_dev;
+  p.plan_checksum = plan_host[PH_CHECKSUM];
+  p.n_units = plan_host[PH_UNITS];
+  p.ws = static_cast<uint8_t*>(workspace);
+  p.status = static_cast<int32_t*>(workspace);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.Sf = final_state;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return KDA_ERR_CUDA;
+  if (launch_simt(p, plan_host[PH_TOTAL_CHUNKS], s) != cudaSuccess) return KDA_ERR_CUDA;
+  return KDA_OK;
+}
+
+extern "C" kda_status_t kda_device_status(const void* workspace, kda_stream_t stream) {
+  if (!workspace) return KDA_ERR_NULL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaMemcpy(&word, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+  if (word == DS_OK) return KDA_OK;
+  if (word == DS_PLAN) return KDA_ERR_PLAN;
+  if (word == DS_TIMEOUT) return KDA_ERR_TIMEOUT;
+  return KDA_ERR_CUDA;
+}

@@ -1,0 +1,61 @@
+// kda_layout.cuh -- kernel parameters and tensor addressing for the three FlashKDA layouts.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "kda_internal.h"
+
+namespace kda {
+
+struct Params {
+  int layout, B, Nqk, Nv, S;
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* g;
+  const __nv_bfloat16* beta;
+  float scale;
+  const float* S0;  // may be null (zero initial state)
+  const float* A_log;
+  const float* dt_bias;
+  float lower_bound;
+  const int32_t* plan;  // device copy
+  int32_t plan_checksum;
+  int n_units;
+  uint8_t* ws;
+  int32_t* status;
+  __nv_bfloat16* out;
+  float* Sf;
+};
+
+// Element offset of the D-vector of (sequence b, head hx of NX heads, token t of the sequence).
+// BNSD [B,NX,S,D], BSND [B,S,NX,D], TND [T,NX,D] with the sequence starting at packed row tok0.
+__device__ __forceinline__ int64_t row_offset(int layout, int NX, int S, int b, int hx, int tok0,
+                                              int t) {
+  if (layout == KDA_LAYOUT_BNSD) return (((int64_t)b * NX + hx) * S + t) * kD;
+  if (layout == KDA_LAYOUT_BSND) return (((int64_t)b * S + t) * NX + hx) * kD;
+  return ((int64_t)(tok0 + t) * NX + hx) * kD;
+}
+
+// Offset of beta for (b, value head h, token t): BNSD [B,Nv,S], BSND [B,S,Nv], TND [T,Nv].
+__device__ __forceinline__ int64_t beta_offset(int layout, int Nv, int S, int b, int h, int tok0,
+                                               int t) {
+  if (layout == KDA_LAYOUT_BNSD) return ((int64_t)b * Nv + h) * S + t;
+  if (layout == KDA_LAYOUT_BSND) return ((int64_t)b * S + t) * Nv + h;
+  return (int64_t)(tok0 + t) * Nv + h;
+}
+
+__device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float x[4]) {
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+  const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+  x[0] = __low2float(a);
+  x[1] = __high2float(a);
+  x[2] = __low2float(c);
+  x[3] = __high2float(c);
+}
+
+cudaError_t launch_simt(const Params& p, int total_chunks, cudaStream_t stream);
+
+}  // namespace kda

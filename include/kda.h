@@ -1,0 +1,140 @@
+/*
+ * kda.h -- C ABI of the B200 chunked Kimi Delta Attention (KDA) prefill library (libkda.so).
+ *
+ * The operation (FlashKDA README, CANNBot-DSL samples/flash_kda, sections 功能说明 and
+ * 参数说明): for every sequence b and value head h, with q/k L2-normalised per row, beta =
+ * sigmoid(beta_logit) and a per-channel log-decay g activated from the raw gate,
+ *
+ *     S_t = S_{t-1} Diag(exp(g_t)) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   S_0 = initial_state
+ *     o_t = scale * S_t q_t
+ *
+ * computed in 64-token chunks (gamma, K~ = gamma*K, K- = K/gamma, Q~ = scale*gamma*Q,
+ * T = stril(diag(beta) K~ K-^T), (I+T)^-1, U, W, then a sequential pass of the state over the
+ * chunks).  The gate activation, whose formula the pages do not print, is
+ *
+ *     g = lower_bound * sigmoid(exp(A_log[h]) * (g_raw + dt_bias[h, :]))     (natural log).
+ *
+ * Calling pattern, mirroring flash_kda_metadata + flash_kda (FlashKDA README, 快速开始):
+ *   1. kda_plan_size + kda_plan on the host: builds an int32 schedule from the shape, the
+ *      layout and the valid lengths only (no tensor values).  Reusable for any call with the
+ *      same shape and lengths (e.g. every layer of a model).
+ *   2. copy the plan to the device; kda_workspace_size; allocate the workspace.
+ *   3. kda_forward: asynchronous, enqueue-only on the given stream.
+ *
+ * Ownership: the caller owns every buffer.  The library never allocates, frees or synchronises
+ * inside kda_forward.  All device pointers must be device memory of the current device.
+ * Errors: every argument check happens on the host before anything is enqueued and is returned
+ * synchronously; nothing is enqueued when a check fails.  Launch failures return KDA_ERR_CUDA.
+ * Device-side problems (a plan that does not match the shape, a bounded wait that gave up) set
+ * a status word in the workspace that kda_device_status reports.  No call traps or aborts.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* kda_stream_t;
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_NULL = 1,        /* a required pointer is NULL */
+  KDA_ERR_LAYOUT = 2,      /* layout is not BNSD, BSND or TND */
+  KDA_ERR_SHAPE = 3,       /* B < 1, S < 1, or a size does not fit the index types */
+  KDA_ERR_HEADS = 4,       /* not 1 <= Nqk <= Nv with Nv % Nqk == 0 */
+  KDA_ERR_DIM = 5,         /* D != 128 */
+  KDA_ERR_LOWER_BOUND = 6, /* lower_bound not in [-5, 0], or scale not finite */
+  KDA_ERR_SEQLENS = 7,     /* cu_seqlens malformed (see kda_plan) */
+  KDA_ERR_PLAN = 8,        /* plan buffer too small, corrupt, or built for another shape */
+  KDA_ERR_ALIAS = 9,       /* initial_state aliases final_state, or out aliases an input */
+  KDA_ERR_WORKSPACE = 10,  /* workspace NULL/too small/not 256-byte aligned */
+  KDA_ERR_CUDA = 11,       /* a CUDA runtime call or a kernel launch failed */
+  KDA_ERR_TIMEOUT = 12,    /* a bounded device-side wait gave up (reported by kda_device_status) */
+  KDA_ERR_DEVICE = 13,     /* the current device is not an sm_100 GPU */
+  KDA_ERR_ALIGN = 14       /* q/k/v/g/out/state/workspace not 16-byte aligned (beta: 2-byte) */
+} kda_status_t;
+
+/* Tensor layouts of q/k/v/g/beta/out (FlashKDA README, 参数说明):
+ *   BNSD: q,k [B,Nqk,S,D]  v,g,out [B,Nv,S,D]  beta [B,Nv,S]
+ *   BSND: q,k [B,S,Nqk,D]  v,g,out [B,S,Nv,D]  beta [B,S,Nv]
+ *   TND : q,k [T,Nqk,D]    v,g,out [T,Nv,D]    beta [T,Nv]     (packed; S field = T)
+ * All tensors are dense and contiguous in the order written. */
+typedef enum { KDA_LAYOUT_BNSD = 0, KDA_LAYOUT_BSND = 1, KDA_LAYOUT_TND = 2 } kda_layout_t;
+
+typedef struct {
+  int32_t layout; /* kda_layout_t */
+  int32_t B;      /* sequences: batch slots (BNSD/BSND) or len(cu_seqlens) - 1 (TND) */
+  int32_t Nqk;    /* query/key heads */
+  int32_t Nv;     /* value heads; value head h reads q/k head h / (Nv / Nqk) */
+  int32_t S;      /* storage length per slot (BNSD/BSND) or total packed tokens T (TND) */
+  int32_t D;      /* head dim, must be 128 (Dk = Dv = D) */
+} kda_shape_t;
+
+/* Chunk length of the method (tokens). */
+#define KDA_CHUNK 64
+
+/* Human-readable name of a status code (static storage, never NULL). */
+KDA_API const char* kda_status_string(kda_status_t status);
+
+/* Number of int32 words kda_plan writes for this shape (header + one record per
+ * (sequence, value head) unit).  Validates the shape. */
+KDA_API kda_status_t kda_plan_size(const kda_shape_t* shape, size_t* n_int32);
+
+/* Build the schedule (the flash_kda_metadata equivalent, FlashKDA README 功能说明: built from
+ * shapes, layout, valid lengths and the device's core count; reads no tensor values).
+ *   cu_seqlens_host: host int32 [B+1] prefix sums of the valid lengths.
+ *     TND : required; cu[0] == 0, cu[B] == T, strictly increasing.
+ *     BNSD/BSND: optional (NULL = every length is S); each length cu[b+1]-cu[b] in [1, S];
+ *     sequence b then occupies storage rows [0, len_b) of slot b (FlashKDA README 约束说明).
+ *   num_sms: multiprocessor count of the target device (>= 1); recorded in the plan.
+ *   plan, n_int32: host output buffer and its capacity in int32 words.
+ * Units are ordered longest first.  Pure host code; never touches the GPU. */
+KDA_API kda_status_t kda_plan(const kda_shape_t* shape, const int32_t* cu_seqlens_host, int32_t num_sms,
+                      int32_t* plan, size_t n_int32);
+
+/* Device workspace bytes kda_forward needs for this plan (host plan).  Always >= 256. */
+KDA_API kda_status_t kda_workspace_size(const int32_t* plan_host, size_t n_int32, size_t* bytes);
+
+/* The forward pass (FlashKDA README, flash_kda): writes out and final_state.
+ *   shape        : as given to kda_plan.
+ *   plan_host    : the plan on the host (read for validation and launch sizing only).
+ *   plan_dev     : the same n_int32 words in device memory (read by the kernels).
+ *   q, k         : bf16 raw queries/keys (normalised in the op).
+ *   v, g         : bf16 values and raw gate.
+ *   beta         : bf16 raw write logits (sigmoid in the op).
+ *   scale        : query scale, usually D^-0.5; must be finite.
+ *   initial_state: fp32 [B,Nv,D(Dv),D(Dk)] or NULL for zeros; read-only.
+ *   A_log        : fp32 [Nv];  dt_bias: fp32 [Nv,D];  lower_bound in [-5, 0].
+ *   workspace    : device scratch of at least kda_workspace_size bytes, 256-byte aligned.
+ *   out          : bf16, v's shape and layout.  Valid rows get the output (rounded to nearest
+ *                  even); rows past a sequence's valid length are written as zeros.
+ *   final_state  : fp32 [B,Nv,D,D]; must not overlap initial_state.
+ * Rows of the inputs past a valid length are never read.  Asynchronous: returns once the
+ * kernels are enqueued on `stream`. */
+KDA_API kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* plan_host,
+                         const int32_t* plan_dev, size_t n_int32, const void* q, const void* k,
+                         const void* v, const void* g, const void* beta, float scale,
+                         const float* initial_state, const float* A_log, const float* dt_bias,
+                         float lower_bound, void* workspace, size_t workspace_bytes, void* out,
+                         float* final_state, kda_stream_t stream);
+
+/* Synchronise `stream` and return the device-side status recorded in `workspace` by the last
+ * kda_forward that used it (KDA_OK, KDA_ERR_PLAN or KDA_ERR_TIMEOUT), or KDA_ERR_CUDA. */
+KDA_API kda_status_t kda_device_status(const void* workspace, kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

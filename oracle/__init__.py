@@ -201,24 +201,19 @@ def _lengths(layout, B, S, cu_seqlens):
     return np.asarray(cu_seqlens, dtype=np.int64)
 
 
-def flash_kda(inp: dict, layout: str, B: int, Nqk: int, Nv: int, S: int, D: int, scale: float,
-              lower_bound: float, cu_seqlens=None, form: str = "chunked", C: int = 64,
-              units=None, threads: int | None = None):
-    """The whole op on raw inputs (bf16 bit arrays + fp32 params), in fp64.
+def run_units(inp: dict, layout: str, B: int, Nqk: int, Nv: int, S: int, D: int, scale: float,
+              lower_bound: float, cu_seqlens=None, units=None, form: str = "chunked", C: int = 64,
+              threads: int | None = None) -> dict:
+    """The op on raw inputs for a list of (b, h) units; returns {(b, h): (out [L, D], S [D, D])}.
 
-    Returns ``(out, final_state, done)``: ``out`` has v's shape (zeros outside the
-    valid rows and for units not computed), ``final_state`` is [B, Nv, D, D] and
-    ``done`` lists the (b, h) units computed.  ``units`` restricts the work to a
-    subset, e.g. a sample of a large workload.
+    ``inp`` holds bf16 bit arrays (q, k, v, g, beta) and fp32 A_log, dt_bias, initial_state.
     """
     cu = _lengths(layout, B, S, cu_seqlens)
     G = Nv // Nqk
     q = inp["q"]; k = inp["k"]; v = inp["v"]; g = inp["g"]; beta = inp["beta"]
     A_log = np.asarray(inp["A_log"], dtype=np.float64)
     dt_bias = np.asarray(inp["dt_bias"], dtype=np.float64)
-    S0 = np.asarray(inp["initial_state"], dtype=np.float64)
-    out = np.zeros(v.shape, dtype=np.float64)
-    fs = np.zeros((B, Nv, D, D), dtype=np.float64)
+    S0 = inp["initial_state"]
     if units is None:
         units = [(b, h) for b in range(B) for h in range(Nv)]
     tnd_cu = cu if layout == "TND" else None
@@ -237,18 +232,35 @@ def flash_kda(inp: dict, layout: str, B: int, Nqk: int, Nv: int, S: int, D: int,
             br = widen_bf16(beta[b, 0:L, h])
         else:
             br = widen_bf16(beta[int(cu[b]):int(cu[b]) + L, h])
-        o, Sf = unit(qr, kr, vr, gr, br, dt_bias[h], A_log[h], lower_bound, scale, S0[b, h],
-                     form=form, C=C)
-        return b, h, L, o, Sf
+        return bh, unit(qr, kr, vr, gr, br, dt_bias[h], A_log[h], lower_bound, scale,
+                        np.asarray(S0[b, h], dtype=np.float64), form=form, C=C)
 
     nthreads = threads or max(1, min(len(units), len(os.sched_getaffinity(0))))
     with ThreadPoolExecutor(max_workers=nthreads) as ex:
-        for b, h, L, o, Sf in ex.map(run, units):
-            if layout == "BNSD":
-                out[b, h, 0:L] = o
-            elif layout == "BSND":
-                out[b, 0:L, h] = o
-            else:
-                out[int(cu[b]):int(cu[b]) + L, h] = o
-            fs[b, h] = Sf
-    return out, fs, list(units)
+        return dict(ex.map(run, units))
+
+
+def flash_kda(inp: dict, layout: str, B: int, Nqk: int, Nv: int, S: int, D: int, scale: float,
+              lower_bound: float, cu_seqlens=None, form: str = "chunked", C: int = 64,
+              units=None, threads: int | None = None):
+    """The whole op on raw inputs (bf16 bit arrays + fp32 params), in fp64.
+
+    Returns ``(out, final_state, done)``: ``out`` has v's shape (zeros outside the
+    valid rows and for units not computed), ``final_state`` is [B, Nv, D, D] and
+    ``done`` lists the (b, h) units computed.
+    """
+    cu = _lengths(layout, B, S, cu_seqlens)
+    res = run_units(inp, layout, B, Nqk, Nv, S, D, scale, lower_bound, cu_seqlens, units, form,
+                    C, threads)
+    out = np.zeros(inp["v"].shape, dtype=np.float64)
+    fs = np.zeros((B, Nv, D, D), dtype=np.float64)
+    for (b, h), (o, Sf) in res.items():
+        L = int(cu[b + 1] - cu[b])
+        if layout == "BNSD":
+            out[b, h, 0:L] = o
+        elif layout == "BSND":
+            out[b, 0:L, h] = o
+        else:
+            out[int(cu[b]):int(cu[b]) + L, h] = o
+        fs[b, h] = Sf
+    return out, fs, list(res.keys())

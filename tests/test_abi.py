@@ -1,0 +1,154 @@
+"""C ABI on the host (no GPU): exports, planner, workspace sizing and argument checks.
+
+The checks follow the FlashKDA README 约束说明: D = 128, B >= 1, S > 0, 1 <= Nqk <= Nv,
+Nv % Nqk == 0, lower_bound in [-5, 0], TND cu_seqlens a strictly increasing prefix sum from 0
+to T, BNSD/BSND valid lengths in [1, S].
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import chunked_kda_prefill_b200 as kda
+from chunked_kda_prefill_b200._lib import KdaShape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+P_I32 = ctypes.POINTER(ctypes.c_int32)
+
+
+@pytest.fixture(scope="module")
+def L():
+    return kda.load()
+
+
+def header_symbols():
+    txt = open(os.path.join(ROOT, "include", "kda.h")).read()
+    return sorted(set(re.findall(r"KDA_API[^;(]*?\b(kda_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_bound_symbols():
+    assert header_symbols() == sorted(kda.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in header_symbols():
+        assert hasattr(L, name), name
+
+
+def _shape(layout=0, B=1, Nqk=1, Nv=1, S=256, D=128):
+    return KdaShape(layout, B, Nqk, Nv, S, D)
+
+
+def _plan(L, shape, cu=None, sms=148):
+    n = ctypes.c_size_t(0)
+    st = L.kda_plan_size(ctypes.byref(shape), ctypes.byref(n))
+    if st:
+        return st, None
+    buf = np.zeros(n.value, dtype=np.int32)
+    cu_p = None
+    if cu is not None:
+        cu = np.asarray(cu, dtype=np.int32)
+        cu_p = cu.ctypes.data_as(P_I32)
+    st = L.kda_plan(ctypes.byref(shape), cu_p, sms, buf.ctypes.data_as(P_I32), buf.size)
+    return st, buf
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=64), 5), (dict(B=0), 3), (dict(S=0), 3), (dict(Nqk=0), 4), (dict(Nqk=3, Nv=2), 4),
+    (dict(Nqk=3, Nv=4), 4), (dict(layout=3), 2), (dict(layout=-1), 2)])
+def test_shape_checks(L, kw, code):
+    st, _ = _plan(L, _shape(**kw))
+    assert st == code
+
+
+@pytest.mark.parametrize("layout,B,S,cu,code", [
+    (2, 2, 100, None, 7),                 # TND needs cu_seqlens
+    (2, 2, 100, [1, 50, 100], 7),         # must start at 0
+    (2, 2, 100, [0, 50, 99], 7),          # must end at T
+    (2, 2, 100, [0, 50, 50, 100], 7),     # (B=2 reads 3 entries) not strictly increasing
+    (2, 2, 100, [0, 100, 100], 7),        # empty sequence
+    (0, 2, 100, [0, 0, 50], 7),           # BNSD length 0
+    (0, 2, 100, [0, 101, 150], 7),        # BNSD length > S
+    (1, 2, 100, [0, 60, 160], 0),         # BSND lengths 60, 100: fine
+    (2, 2, 100, [0, 37, 100], 0),
+])
+def test_seqlen_checks(L, layout, B, S, cu, code):
+    st, _ = _plan(L, _shape(layout=layout, B=B, S=S, Nqk=2, Nv=4), cu)
+    assert st == code
+
+
+def test_plan_records_longest_first(L):
+    cu = [0, 10, 200, 265]
+    st, p = _plan(L, _shape(layout=2, B=3, Nqk=1, Nv=2, S=265), cu)
+    assert st == 0
+    assert p[0] == 0x4B444131 and p[4] == 6 and p[11] == (3 + 2 + 1) * 2 and p[12] == 3
+    recs = p[16:].reshape(6, 8)
+    # (b, h, hq, tok_start, len, chunks, chunk_offset)
+    assert [tuple(r[:7]) for r in recs] == [
+        (1, 0, 0, 10, 190, 3, 0), (1, 1, 0, 10, 190, 3, 3), (2, 0, 0, 200, 65, 2, 6),
+        (2, 1, 0, 200, 65, 2, 8), (0, 0, 0, 0, 10, 1, 10), (0, 1, 0, 0, 10, 1, 11)]
+    ws = ctypes.c_size_t(0)
+    assert L.kda_workspace_size(p.ctypes.data_as(P_I32), p.size, ctypes.byref(ws)) == 0
+    assert ws.value >= 256
+
+
+def test_plan_gqa_head_map(L):
+    st, p = _plan(L, _shape(layout=0, B=1, Nqk=4, Nv=16, S=64))
+    recs = p[16:].reshape(16, 8)
+    assert [int(r[2]) for r in recs] == [h // 4 for h in range(16)]
+
+
+def test_plan_capacity_and_corruption(L):
+    sh = _shape(layout=0, B=2, Nqk=2, Nv=2, S=300)
+    n = ctypes.c_size_t(0)
+    assert L.kda_plan_size(ctypes.byref(sh), ctypes.byref(n)) == 0
+    small = np.zeros(n.value - 1, dtype=np.int32)
+    assert L.kda_plan(ctypes.byref(sh), None, 148, small.ctypes.data_as(P_I32), small.size) == 8
+    st, p = _plan(L, sh)
+    ws = ctypes.c_size_t(0)
+    bad = p.copy()
+    bad[16 + 4] += 1  # edit a record: the checksum no longer matches
+    assert L.kda_workspace_size(bad.ctypes.data_as(P_I32), bad.size, ctypes.byref(ws)) == 8
+    assert L.kda_workspace_size(p.ctypes.data_as(P_I32), p.size - 1, ctypes.byref(ws)) == 8
+
+
+def _fwd(L, shape, plan, **over):
+    """kda_forward with fake (never dereferenced) device pointers; every check is on the host."""
+    a = dict(q=0x10000000, k=0x20000000, v=0x30000000, g=0x40000000, beta=0x50000000,
+             scale=0.088, S0=0x60000000, A_log=0x70000000, dt=0x71000000, lb=-5.0,
+             ws=0x80000000, ws_bytes=1 << 40, out=0x90000000, fs=0xA0000000, plan_dev=0xB0000000)
+    a.update(over)
+    return L.kda_forward(ctypes.byref(shape), plan.ctypes.data_as(P_I32), a["plan_dev"],
+                         plan.size, a["q"], a["k"], a["v"], a["g"], a["beta"], a["scale"],
+                         a["S0"], a["A_log"], a["dt"], a["lb"], a["ws"], a["ws_bytes"], a["out"],
+                         a["fs"], None)
+
+
+def test_forward_argument_checks(L):
+    sh = _shape(layout=0, B=1, Nqk=1, Nv=1, S=256)
+    st, p = _plan(L, sh)
+    assert st == 0
+    assert _fwd(L, sh, p, q=None) == 1
+    assert _fwd(L, sh, p, out=None) == 1
+    assert _fwd(L, sh, p, lb=0.5) == 6
+    assert _fwd(L, sh, p, lb=-5.01) == 6
+    assert _fwd(L, sh, p, lb=float("nan")) == 6
+    assert _fwd(L, sh, p, scale=float("inf")) == 6
+    assert _fwd(L, sh, p, ws_bytes=100) == 10
+    assert _fwd(L, sh, p, ws=0x80000010) == 10          # not 256-byte aligned
+    assert _fwd(L, sh, p, fs=0x60000000) == 9           # final_state aliases initial_state
+    assert _fwd(L, sh, p, out=0x30000000 + 64) == 9     # out overlaps v
+    assert _fwd(L, sh, p, q=0x10000008) == 14           # q not 16-byte aligned
+    assert _fwd(L, sh, p, beta=0x50000001) == 14        # beta not 2-byte aligned
+    other = _shape(layout=0, B=1, Nqk=1, Nv=1, S=512)
+    assert _fwd(L, other, p) == 8                       # plan built for another shape
+    # all host checks pass: what remains needs a GPU (no device here -> CUDA/device error)
+    assert _fwd(L, sh, p) in (11, 13)
+
+
+def test_status_strings(L):
+    for code in range(15):
+        s = L.kda_status_string(code).decode()
+        assert s.startswith("KDA_")
