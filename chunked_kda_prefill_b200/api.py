@@ -152,6 +152,34 @@ def flash_kda(q, k, v, g, beta, scale: float, initial_state, A_log, dt_bias, low
     return out, final_state
 
 
+def flash_kda_noalloc(q, k, v, g, beta, scale: float, initial_state, A_log, dt_bias,
+                      lower_bound: float, layout: str, plan: KdaPlan, out: torch.Tensor,
+                      final_state: torch.Tensor, stream: torch.cuda.Stream | None = None):
+    """flash_kda through kda_forward_noalloc: no workspace, the library's fixed scratch instead.
+
+    For callers that cannot allocate device memory; the caller still provides out and
+    final_state.  Raises KdaError(KDA_ERR_CAPACITY) for problems larger than the scratch.
+    """
+    dev = q.device
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (out, "out")):
+        _expect(t, name, torch.bfloat16, dev)
+    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias"), (final_state, "final_state")):
+        _expect(t, name, torch.float32, dev)
+    if initial_state is not None:
+        _expect(initial_state, "initial_state", torch.float32, dev)
+    if plan.layout != layout:
+        raise KdaError(8, "plan was built for another layout")
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    code = _lib.load().kda_forward_noalloc(
+        ctypes.byref(plan.shape), plan.host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+        plan.dev.data_ptr(), plan.host.size, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+        g.data_ptr(), beta.data_ptr(), float(scale), _ptr(initial_state), A_log.data_ptr(),
+        dt_bias.data_ptr(), float(lower_bound), out.data_ptr(), final_state.data_ptr(),
+        s.cuda_stream)
+    check(code, "kda_forward_noalloc")
+    return out, final_state
+
+
 def device_status(workspace: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
     """Synchronise and raise if the last forward on this workspace recorded a device error."""
     s = stream if stream is not None else torch.cuda.current_stream(workspace.device)

@@ -78,6 +78,9 @@ extern "C" const char* kda_status_string(kda_status_t st) {
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device-side wait gave up";
     case KDA_ERR_DEVICE: return "KDA_ERR_DEVICE: current device is not an sm_100 GPU";
     case KDA_ERR_ALIGN: return "KDA_ERR_ALIGN: tensor base pointers must be 16-byte aligned";
+    case KDA_ERR_CAPACITY:
+      return "KDA_ERR_CAPACITY: problem needs more scratch than kda_forward_noalloc's fixed "
+             "KDA_NOALLOC_SCRATCH_BYTES; use kda_forward with a workspace";
   }
   return "KDA_ERR_UNKNOWN";
 }

@@ -1,0 +1,72 @@
+// kda_noalloc.cu -- kda_forward_noalloc: the forward pass for callers that cannot allocate.
+//
+// Some callers have no way to provide the device workspace kda_forward needs:
+// - a plugin interface that hands the library only its input and output tensors;
+// - a host runtime that owns every device byte through its own pool and forbids extra
+//   cudaMalloc calls (cudaMalloc can also synchronise the device, which some schedulers must
+//   avoid).
+// For them the library keeps one fixed scratch region per GPU: a file-scope static __device__
+// array of KDA_NOALLOC_SCRATCH_BYTES. Every GPU that loads the library holds it until the
+// process exits. The entry point calls no cudaMalloc, cudaFree or allocating library routine.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "kda_internal.h"
+
+namespace {
+
+// The scratch itself.  In host code this name is only a host-side stand-in for the symbol, not a
+// device address; the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_kda_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_dev_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch on the current device, looked up once per device (with that
+// device current) on the first call and cached.
+kda_status_t scratch_on_current_device(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_dev_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_kda_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) return KDA_ERR_CUDA;
+    g_scratch_dev_ptr[dev] = ptr;
+  }
+  *out = g_scratch_dev_ptr[dev];
+  return KDA_OK;
+}
+
+}  // namespace
+
+using namespace kda;
+
+extern "C" kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int32_t* plan_host,
+                                            const int32_t* plan_dev, size_t n_int32,
+                                            const void* q, const void* k, const void* v,
+                                            const void* g, const void* beta, float scale,
+                                            const float* initial_state, const float* A_log,
+                                            const float* dt_bias, float lower_bound, void* out,
+                                            float* final_state, kda_stream_t stream) {
+  kda_status_t st = validate_shape(shape);
+  if (st != KDA_OK) return st;
+  if (!plan_host) return KDA_ERR_NULL;
+  st = validate_plan(plan_host, n_int32, shape);
+  if (st != KDA_OK) return st;
+  size_t need = 0;
+  st = kda_workspace_size(plan_host, n_int32, &need);
+  if (st != KDA_OK) return st;
+  if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_CAPACITY;
+  void* scratch = nullptr;
+  st = scratch_on_current_device(&scratch);
+  if (st != KDA_OK) return st;
+  // The status word at the start of the scratch is cleared by kda_forward on every call; every
+  // other byte the kernels read is written earlier in the same call.
+  return kda_forward(shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale, initial_state,
+                     A_log, dt_bias, lower_bound, scratch, (size_t)KDA_NOALLOC_SCRATCH_BYTES, out,
+                     final_state, stream);
+}

@@ -62,7 +62,8 @@ typedef enum {
   KDA_ERR_CUDA = 11,       /* a CUDA runtime call or a kernel launch failed */
   KDA_ERR_TIMEOUT = 12,    /* a bounded device-side wait gave up (reported by kda_device_status) */
   KDA_ERR_DEVICE = 13,     /* the current device is not an sm_100 GPU */
-  KDA_ERR_ALIGN = 14       /* q/k/v/g/out/state/workspace not 16-byte aligned (beta: 2-byte) */
+  KDA_ERR_ALIGN = 14,      /* q/k/v/g/out/state/workspace not 16-byte aligned (beta: 2-byte) */
+  KDA_ERR_CAPACITY = 15    /* kda_forward_noalloc: problem needs more than its fixed scratch */
 } kda_status_t;
 
 /* Tensor layouts of q/k/v/g/beta/out (FlashKDA README, 参数说明):
@@ -132,6 +133,36 @@ KDA_API kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* plan_h
 /* Synchronise `stream` and return the device-side status recorded in `workspace` by the last
  * kda_forward that used it (KDA_OK, KDA_ERR_PLAN or KDA_ERR_TIMEOUT), or KDA_ERR_CUDA. */
 KDA_API kda_status_t kda_device_status(const void* workspace, kda_stream_t stream);
+
+/* Bytes of the fixed, library-owned scratch that kda_forward_noalloc uses on each GPU. */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* kda_forward for callers that cannot allocate device memory.  The pages have no counterpart
+ * of this call; it exists for callers that cannot provide a device workspace: a plugin
+ * interface that hands over only the tensors, or a host runtime whose memory pool forbids
+ * extra cudaMalloc calls (cudaMalloc can also synchronise the device).
+ *
+ * Arguments, layouts and results are those of kda_forward, without workspace and
+ * workspace_bytes.  Instead the library uses one fixed scratch array of
+ * KDA_NOALLOC_SCRATCH_BYTES per GPU: a static __device__ array that every GPU loading libkda.so
+ * holds until the process exits.  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *   - Problems whose kda_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES are rejected with
+ *     KDA_ERR_CAPACITY before anything is enqueued (the current kernels need 148,480 bytes per
+ *     64-token chunk of every (sequence, value head), plus 256, so at most 451 such chunks).
+ *   - The first call on each device looks up the scratch's device address with that device
+ *     current and caches it; make that first call before any stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the last call's contents
+ *     (the call clears what must start at zero).  Calls whose kernels overlap on the GPU (two
+ *     streams, or two host threads) race on it: serialise them.
+ *   - The device status word lives in that scratch; there is no kda_device_status for it. */
+KDA_API kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int32_t* plan_host,
+                                         const int32_t* plan_dev, size_t n_int32, const void* q,
+                                         const void* k, const void* v, const void* g,
+                                         const void* beta, float scale,
+                                         const float* initial_state, const float* A_log,
+                                         const float* dt_bias, float lower_bound, void* out,
+                                         float* final_state, kda_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -149,6 +149,6 @@ def test_forward_argument_checks(L):
 
 
 def test_status_strings(L):
-    for code in range(15):
+    for code in range(16):
         s = L.kda_status_string(code).decode()
         assert s.startswith("KDA_")
