@@ -188,8 +188,8 @@ def device_status(workspace: torch.Tensor, stream: torch.cuda.Stream | None = No
 
 def kernels_per_forward() -> int:
     """Kernels of this library that one kda_forward launches."""
-    return 2
+    return 1
 
 
 def forward_kernel_names() -> str:
-    return "kda_chunk_simt_kernel + kda_scan_simt_kernel"
+    return "kda_fused_kernel"

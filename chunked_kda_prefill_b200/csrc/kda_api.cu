@@ -36,17 +36,17 @@ kda_status_t check_device() {
 }
 
 }  // namespace
-}  // namespace kda
 
-using namespace kda;
+size_t simt_workspace_bytes(const int32_t* plan) {
+  return kWsHeaderBytes + (size_t)plan[PH_TOTAL_CHUNKS] * kWsChunkBytes;
+}
 
-extern "C" kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* plan_host,
-                                    const int32_t* plan_dev, size_t n_int32, const void* q,
-                                    const void* k, const void* v, const void* g, const void* beta,
-                                    float scale, const float* initial_state, const float* A_log,
-                                    const float* dt_bias, float lower_bound, void* workspace,
-                                    size_t workspace_bytes, void* out, float* final_state,
-                                    kda_stream_t stream) {
+kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* plan_host,
+                          const int32_t* plan_dev, size_t n_int32, const void* q, const void* k,
+                          const void* v, const void* g, const void* beta, float scale,
+                          const float* initial_state, const float* A_log, const float* dt_bias,
+                          float lower_bound, void* workspace, size_t workspace_bytes, void* out,
+                          float* final_state, cudaStream_t stream, float* dbg) {
   kda_status_t st = validate_shape(shape);
   if (st != KDA_OK) return st;
   if (!plan_host || !plan_dev || !q || !k || !v || !g || !beta || !A_log || !dt_bias ||
@@ -56,16 +56,13 @@ extern "C" kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* pla
   if (st != KDA_OK) return st;
   if (!std::isfinite(scale)) return KDA_ERR_LOWER_BOUND;
   if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_LOWER_BOUND;
-
   {
     const void* a16[] = {q, k, v, g, out, final_state, A_log, dt_bias, plan_dev, initial_state};
     for (const void* ptr : a16)
       if (reinterpret_cast<uintptr_t>(ptr) & 15u) return KDA_ERR_ALIGN;
     if (reinterpret_cast<uintptr_t>(beta) & 1u) return KDA_ERR_ALIGN;
   }
-  size_t need = 0;
-  st = kda_workspace_size(plan_host, n_int32, &need);
-  if (st != KDA_OK) return st;
+  const size_t need = (path == PATH_SIMT) ? simt_workspace_bytes(plan_host) : kWsHeaderBytes;
   if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return KDA_ERR_WORKSPACE;
 
@@ -114,10 +111,62 @@ extern "C" kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* pla
   p.out = static_cast<__nv_bfloat16*>(out);
   p.Sf = final_state;
 
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return KDA_ERR_CUDA;
-  if (launch_simt(p, plan_host[PH_TOTAL_CHUNKS], s) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, 4, stream) != cudaSuccess) return KDA_ERR_CUDA;
+  const cudaError_t e = (path == PATH_SIMT) ? launch_simt(p, plan_host[PH_TOTAL_CHUNKS], stream)
+                                            : launch_fused(p, dbg, stream);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* plan_host,
+                                    const int32_t* plan_dev, size_t n_int32, const void* q,
+                                    const void* k, const void* v, const void* g, const void* beta,
+                                    float scale, const float* initial_state, const float* A_log,
+                                    const float* dt_bias, float lower_bound, void* workspace,
+                                    size_t workspace_bytes, void* out, float* final_state,
+                                    kda_stream_t stream) {
+  return forward_impl(PATH_FUSED, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
+                      initial_state, A_log, dt_bias, lower_bound, workspace, workspace_bytes, out,
+                      final_state, reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+// ---- internal entry points for the GPU tests (not part of include/kda.h) ----
+
+// The two-kernel fp32 CUDA-core path, with a caller workspace of kda_simt_workspace_size bytes.
+extern "C" __attribute__((visibility("default"))) kda_status_t kda_forward_simt(
+    const kda_shape_t* shape, const int32_t* plan_host, const int32_t* plan_dev, size_t n_int32,
+    const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+    const float* initial_state, const float* A_log, const float* dt_bias, float lower_bound,
+    void* workspace, size_t workspace_bytes, void* out, float* final_state, kda_stream_t stream) {
+  return forward_impl(PATH_SIMT, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
+                      initial_state, A_log, dt_bias, lower_bound, workspace, workspace_bytes, out,
+                      final_state, reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+extern "C" __attribute__((visibility("default"))) kda_status_t kda_simt_workspace_size(
+    const int32_t* plan_host, size_t n_int32, size_t* bytes) {
+  if (!bytes) return KDA_ERR_NULL;
+  const kda_status_t st = validate_plan(plan_host, n_int32, nullptr);
+  if (st != KDA_OK) return st;
+  *bytes = simt_workspace_bytes(plan_host);
   return KDA_OK;
+}
+
+// The fused path with every chunk's intermediates (W, U, Q~, K^, Aqk, gamma_last; fp32, the
+// two-kernel workspace layout after its 256-byte header) written to `dump`.
+extern "C" __attribute__((visibility("default"))) kda_status_t kda_forward_debug(
+    const kda_shape_t* shape, const int32_t* plan_host, const int32_t* plan_dev, size_t n_int32,
+    const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+    const float* initial_state, const float* A_log, const float* dt_bias, float lower_bound,
+    void* workspace, size_t workspace_bytes, void* out, float* final_state, float* dump,
+    kda_stream_t stream) {
+  if (!dump) return KDA_ERR_NULL;
+  return forward_impl(PATH_FUSED, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
+                      initial_state, A_log, dt_bias, lower_bound, workspace, workspace_bytes, out,
+                      final_state, reinterpret_cast<cudaStream_t>(stream), dump);
 }
 
 extern "C" kda_status_t kda_device_status(const void* workspace, kda_stream_t stream) {

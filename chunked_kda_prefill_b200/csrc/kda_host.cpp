@@ -176,6 +176,6 @@ extern "C" kda_status_t kda_workspace_size(const int32_t* plan, size_t n, size_t
   if (!bytes) return KDA_ERR_NULL;
   kda_status_t st = validate_plan(plan, n, nullptr);
   if (st != KDA_OK) return st;
-  *bytes = kWsHeaderBytes + (size_t)plan[PH_TOTAL_CHUNKS] * kWsChunkBytes;
+  *bytes = kWsHeaderBytes;  // the fused kernel keeps only its status word in the workspace
   return KDA_OK;
 }

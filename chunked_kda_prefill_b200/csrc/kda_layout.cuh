@@ -56,6 +56,24 @@ __device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float x[4]) {
   x[3] = __high2float(c);
 }
 
+// The two-kernel fp32 CUDA-core path (kda_simt.cu): needs kWsHeaderBytes + total_chunks *
+// kWsChunkBytes of workspace.
 cudaError_t launch_simt(const Params& p, int total_chunks, cudaStream_t stream);
+// The fused tcgen05 path (kda_fused.cu): needs kWsHeaderBytes of workspace.  A non-null `dbg`
+// receives every chunk's intermediates in the two-kernel workspace layout (test aid).
+cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream);
+
+enum ForwardPath : int { PATH_FUSED = 0, PATH_SIMT = 1 };
+
+// Shared body of the forward entry points: every host check, then the launches of `path`.
+kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* plan_host,
+                          const int32_t* plan_dev, size_t n_int32, const void* q, const void* k,
+                          const void* v, const void* g, const void* beta, float scale,
+                          const float* initial_state, const float* A_log, const float* dt_bias,
+                          float lower_bound, void* workspace, size_t workspace_bytes, void* out,
+                          float* final_state, cudaStream_t stream, float* dbg);
+
+// Workspace bytes of the two-kernel path for a validated plan.
+size_t simt_workspace_bytes(const int32_t* plan);
 
 }  // namespace kda

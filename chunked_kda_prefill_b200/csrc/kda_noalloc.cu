@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "kda_internal.h"
+#include "kda_layout.cuh"
 
 namespace {
 
@@ -57,16 +58,16 @@ extern "C" kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int3
   if (!plan_host) return KDA_ERR_NULL;
   st = validate_plan(plan_host, n_int32, shape);
   if (st != KDA_OK) return st;
-  size_t need = 0;
-  st = kda_workspace_size(plan_host, n_int32, &need);
-  if (st != KDA_OK) return st;
+  const size_t need = simt_workspace_bytes(plan_host);
   if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_CAPACITY;
   void* scratch = nullptr;
   st = scratch_on_current_device(&scratch);
   if (st != KDA_OK) return st;
-  // The status word at the start of the scratch is cleared by kda_forward on every call; every
-  // other byte the kernels read is written earlier in the same call.
-  return kda_forward(shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale, initial_state,
-                     A_log, dt_bias, lower_bound, scratch, (size_t)KDA_NOALLOC_SCRATCH_BYTES, out,
-                     final_state, stream);
+  // The two-kernel path: the per-chunk intermediates live in the scratch.  The status word at
+  // its start is cleared on every call; every other byte the kernels read is written earlier in
+  // the same call.
+  return forward_impl(PATH_SIMT, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
+                      initial_state, A_log, dt_bias, lower_bound, scratch,
+                      (size_t)KDA_NOALLOC_SCRATCH_BYTES, out, final_state,
+                      reinterpret_cast<cudaStream_t>(stream), nullptr);
 }

@@ -73,12 +73,12 @@ def test_small_cases_parity(case, cuda_ok):
     check_full(w, inp)
 
 
-def test_long_memory_stress(cuda_ok):
-    """lower_bound = 0 (no decay) over 4 chunks and -0.1 over 128 chunks: errors would pile up."""
-    for lb, S in ((0.0, 256), (-0.1, 8192)):
-        w = W.custom(f"stress{lb}", "BNSD", 1, 1, 1, S, [S], lower_bound=lb, init_state="normal",
-                     seed=23)
-        check_full(w, W.generate(w))
+@pytest.mark.parametrize("lb,S", [(0.0, 256), (0.0, 2048), (-0.1, 8192)])
+def test_long_memory_stress(lb, S, cuda_ok):
+    """No decay (lower_bound = 0) and slow decay over many chunks: rounding would pile up."""
+    w = W.custom(f"stress{lb}_{S}", "BNSD", 1, 1, 1, S, [S], lower_bound=lb,
+                 init_state="normal", seed=23)
+    check_full(w, W.generate(w))
 
 
 def _same(a, b):

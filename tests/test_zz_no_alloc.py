@@ -41,10 +41,10 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_ok):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_ok):
-    w = W.workload(3)  # 1712 chunks: more than the fixed scratch holds
+    w = W.workload(3)  # 1712 chunk-heads: more than the fixed scratch holds
     shape = kda.KdaShape(1, w.B, w.Nqk, w.Nv, w.S, w.D)
     plan = kda.make_plan(shape, w.layout, w.cu_seqlens, device="cuda")
-    assert plan.workspace_bytes > (64 << 20)
+    assert 256 + plan.total_chunks * 148480 > (64 << 20)
     x = torch.zeros(1, dtype=torch.bfloat16, device="cuda")
     f = torch.zeros(1, dtype=torch.float32, device="cuda")
     with pytest.raises(kda.KdaError) as e:
