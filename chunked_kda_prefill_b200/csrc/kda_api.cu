@@ -46,7 +46,8 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
                           const void* v, const void* g, const void* beta, float scale,
                           const float* initial_state, const float* A_log, const float* dt_bias,
                           float lower_bound, void* workspace, size_t workspace_bytes, void* out,
-                          float* final_state, cudaStream_t stream, float* dbg) {
+                          float* final_state, cudaStream_t stream, float* dbg,
+                          unsigned long long* tprof) {
   kda_status_t st = validate_shape(shape);
   if (st != KDA_OK) return st;
   if (!plan_host || !plan_dev || !q || !k || !v || !g || !beta || !A_log || !dt_bias ||
@@ -110,6 +111,7 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   p.status = static_cast<int32_t*>(workspace);
   p.out = static_cast<__nv_bfloat16*>(out);
   p.Sf = final_state;
+  p.tprof = tprof;
 
   if (cudaMemsetAsync(workspace, 0, 4, stream) != cudaSuccess) return KDA_ERR_CUDA;
   const cudaError_t e = (path == PATH_SIMT) ? launch_simt(p, plan_host[PH_TOTAL_CHUNKS], stream)
@@ -156,17 +158,18 @@ extern "C" __attribute__((visibility("default"))) kda_status_t kda_simt_workspac
 }
 
 // The fused path with every chunk's intermediates (W, U, Q~, K^, Aqk, gamma_last; fp32, the
-// two-kernel workspace layout after its 256-byte header) written to `dump`.
+// two-kernel workspace layout after its 256-byte header) written to `dump` (if not NULL), and
+// CTA 0's clock64() at each phase boundary of its first 64 chunks written to `tprof` (if not
+// NULL; 16 words per chunk).
 extern "C" __attribute__((visibility("default"))) kda_status_t kda_forward_debug(
     const kda_shape_t* shape, const int32_t* plan_host, const int32_t* plan_dev, size_t n_int32,
     const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
     const float* initial_state, const float* A_log, const float* dt_bias, float lower_bound,
     void* workspace, size_t workspace_bytes, void* out, float* final_state, float* dump,
-    kda_stream_t stream) {
-  if (!dump) return KDA_ERR_NULL;
+    unsigned long long* tprof, kda_stream_t stream) {
   return forward_impl(PATH_FUSED, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
                       initial_state, A_log, dt_bias, lower_bound, workspace, workspace_bytes, out,
-                      final_state, reinterpret_cast<cudaStream_t>(stream), dump);
+                      final_state, reinterpret_cast<cudaStream_t>(stream), dump, tprof);
 }
 
 extern "C" kda_status_t kda_device_status(const void* workspace, kda_stream_t stream) {

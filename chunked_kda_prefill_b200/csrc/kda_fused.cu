@@ -59,7 +59,9 @@ constexpr uint32_t OFF_Q = 0, OFF_K = 16384, OFF_G = 32768, OFF_V = 49152;
 constexpr uint32_t SM_AOP = 131072;   // [128 rows][128] bf16, 2 atoms of 16 KB; after phase 2:
 constexpr uint32_t SM_KLO = SM_AOP;           //   K^ lo part [64][128] (16 KB)
 constexpr uint32_t SM_XWLO = SM_AOP + 16384;  //   Xsol lo part [64][64], then -W lo part [64][128]
-constexpr uint32_t SM_BT = 163840;    // B^(0..3): 16,32,48,64 rows; reused by the solve
+constexpr uint32_t SM_OSTG = SM_AOP;          //   phase 8: out tile [64 tokens][128] for the TMA store
+constexpr uint32_t SM_BT = 163840;    // [B^(0); B^(1); B^(2); B^(3)]: one 160-row tile; then the solve
+constexpr uint32_t BT_ROWS = 160;
 constexpr uint32_t SM_XSOL = 204800;  // [64][64] bf16
 constexpr uint32_t SM_AQK = 212992;   // [64][64] bf16
 constexpr uint32_t SM_WTOT = 221184;  // fp32 [8][128] warp totals of the gate cumsum
@@ -72,7 +74,12 @@ constexpr uint32_t SM_FLAG = 228132;
 constexpr uint32_t SM_END = 228160;
 constexpr size_t kFusedSmemBytes = SM_END + 1024;
 
-__device__ __forceinline__ uint32_t btoff(int I) { return 2048u * I * (I + 1); }
+// Phase timestamps for performance analysis (CTA 0, thread 0, first 64 chunks).
+#define KDA_TS(slot_)                                                        \
+  do {                                                                       \
+    if (tprof_on) p.tprof[(size_t)gidx * 32 + (slot_)] = clock64();          \
+  } while (0)
+
 __device__ __forceinline__ uint32_t dcol(int I) { return 8u * I * (I + 1); }
 
 __device__ __forceinline__ bool plan_ok(const Params& p) {
@@ -96,14 +103,30 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct Maps {
-  CUtensorMap q, k, v, g;
+  CUtensorMap q, k, v, g, o;
 };
 
-// TMA of chunk c of unit u into ring slot `slot` (all four tensors, two 64-column boxes each).
-__device__ void issue_chunk_loads(const Params& p, const Maps& m, uint32_t sbase, int u, int c,
-                                  int slot) {
-  const int32_t* rec = p.plan + kPlanHeader + u * kPlanRecord;
-  const int b = rec[PR_B], h = rec[PR_H], hq = rec[PR_HQ], tok0 = rec[PR_TOK_START];
+// A unit's plan record as the producer keeps it in registers.
+struct UnitRec {
+  int b, h, hq, tok0, nch;
+};
+__device__ __forceinline__ UnitRec read_rec(const Params& p, int u) {
+  UnitRec r{0, 0, 0, 0, 0};
+  if (u < p.n_units) {
+    const int32_t* rec = p.plan + kPlanHeader + u * kPlanRecord;
+    r.b = rec[PR_B];
+    r.h = rec[PR_H];
+    r.hq = rec[PR_HQ];
+    r.tok0 = rec[PR_TOK_START];
+    r.nch = rec[PR_CHUNKS];
+  }
+  return r;
+}
+
+// TMA of chunk c of unit `ur` into ring slot `slot` (all four tensors, two 64-column boxes each).
+__device__ void issue_chunk_loads(const Params& p, const Maps& m, uint32_t sbase, const UnitRec& ur,
+                                  int c, int slot) {
+  const int b = ur.b, h = ur.h, hq = ur.hq, tok0 = ur.tok0;
   const uint32_t bar = sbase + SM_BAR + 8u * slot;
   const uint32_t dst = sbase + slot * SLOT_BYTES;
   mbar_arrive_expect_tx(bar, SLOT_BYTES);
@@ -121,6 +144,45 @@ __device__ void issue_chunk_loads(const Params& p, const Maps& m, uint32_t sbase
     tma_load_3d(dst + OFF_K + a * 8192, &m.k, bar, 64 * a, qc1, qc2);
     tma_load_3d(dst + OFF_G + a * 8192, &m.g, bar, 64 * a, vc1, vc2);
     tma_load_3d(dst + OFF_V + a * 8192, &m.v, bar, 64 * a, vc1, vc2);
+  }
+}
+
+// Rows of D_BLK (row block BLK of the intra product) -> T (fp32, scaled by beta, strictly
+// lower, into Ts with pitch 68) for k rows, or Aqk (bf16, lower with diagonal, K-major) for
+// q rows.  The TMEM load is issued by the whole warp; only lanes in row block BLK write.
+template <int BLK>
+__device__ __forceinline__ void extract_block(uint32_t ta, int r, bool krow, float br, float* Ts,
+                                              uint8_t* aqk) {
+  constexpr int NC = BLK + 1;
+  constexpr int TP = 68;
+  uint32_t v[16 * NC];
+#pragma unroll
+  for (int ch = 0; ch < NC; ++ch)
+    tmem_ld16(ta + 8u * BLK * (BLK + 1) + 16 * ch, *reinterpret_cast<uint32_t(*)[16]>(v + 16 * ch));
+  tmem_wait_ld();
+  if ((r >> 4) != BLK) return;
+  if (krow) {
+#pragma unroll
+    for (int s0 = 0; s0 < 64; s0 += 4) {
+      float f[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int s = s0 + e;
+        f[e] = (s < 16 * NC && s < r) ? br * __uint_as_float(v[s < 16 * NC ? s : 0]) : 0.f;
+      }
+      *reinterpret_cast<float4*>(Ts + r * TP + s0) = make_float4(f[0], f[1], f[2], f[3]);
+    }
+  } else {
+#pragma unroll
+    for (int s0 = 0; s0 < 64; s0 += 8) {
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int s = s0 + e;
+        f[e] = (s < 16 * NC && s <= r) ? __uint_as_float(v[s < 16 * NC ? s : 0]) : 0.f;
+      }
+      *reinterpret_cast<uint4*>(aqk + sw128_offset(64, r, s0)) = pack8(f);
+    }
   }
 }
 
@@ -167,19 +229,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int G_stride = gridDim.x;
   // producer cursor (thread 0): next (unit, chunk) of this CTA's stream to load
+  // (plan records are read one unit ahead so no global load sits on the issue path)
   int pu = blockIdx.x, pc = 0;
   uint32_t issued = 0;
+  UnitRec prec{0, 0, 0, 0, 0}, nrec{0, 0, 0, 0, 0};
   auto produce = [&]() {
     if (pu >= p.n_units) return;
-    issue_chunk_loads(p, maps, sbase, pu, pc, issued & 1);
+    issue_chunk_loads(p, maps, sbase, prec, pc, issued & 1);
     ++issued;
-    const int nch = p.plan[kPlanHeader + pu * kPlanRecord + PR_CHUNKS];
-    if (++pc == nch) {
+    if (++pc == prec.nch) {
       pc = 0;
       pu += G_stride;
+      prec = nrec;
+      nrec = read_rec(p, pu + G_stride);
     }
   };
   if (tid == 0) {
+    prec = read_rec(p, pu);
+    nrec = read_rec(p, pu + G_stride);
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.k);
     tma_prefetch_desc(&maps.v);
@@ -265,6 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t0 = c * kChunk;
       const int n = min(kChunk, L - t0);
       const bool last = (c == nch - 1);
+      const bool tprof_on = p.tprof && blockIdx.x == 0 && tid == 0 && gidx < 64;
+      KDA_TS(0);
 
       // =================== phase 1: prologue and operand tiles ===================
       const float blog = bl_next;  // this chunk's beta logit (row tid), loaded one chunk ahead
@@ -272,13 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         bl_next = __bfloat162float(
             p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t0 + kChunk + tid)]);
       if (!mbar_wait_bounded(sbase + SM_BAR + 8u * slot, (gidx >> 1) & 1u, kWaitLimit)) fail();
+      if (tid == 0) tma_store_wait_read();  // the out tile staged in the Aop region was read
+      KDA_TS(1);
 
       float G[4][8];
       uint4 khlo[4];  // K^ lo parts of this thread's rows, stored once the intra MMA is done
       {
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        // g_act * log2(e) = lb log2(e) / (1 + 2^(-log2(e) e^A_log (g_raw + dt_bias)))
+        const float ca = -a_h * kLog2e;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = r0 + i;
@@ -286,12 +356,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           unpack8(*reinterpret_cast<const uint4*>(sG + sw128_offset(64, r, j0)), gv);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float z = a_h * (gv[e] + dtb[e]);
-            const float s = __fdividef(1.0f, 1.0f + __expf(-z));
-            acc[e] += (r < n) ? lbl2 * s : 0.0f;
-            G[i][e] = acc[e];
+            const float sg = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
+            G[i][e] = (r < n) ? sg : 0.0f;
           }
         }
+#pragma unroll
+        for (int i = 1; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) G[i][e] += G[i - 1][e];
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -308,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (tid < kChunk) beta_s[tid] = (tid < n) ? __fdividef(1.0f, 1.0f + __expf(-blog)) : 0.0f;
       __syncthreads();
+      KDA_TS(11);
       {
         float pre[8];
 #pragma unroll
@@ -327,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         dst[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
       }
       __syncthreads();
+      KDA_TS(12);
       if (tid < kD) gcs[tid] = ex2(refg[3 * kD + tid]);
       {
         // reference rows of this thread's 16-row block Jb (read straight from shared memory so
@@ -346,26 +420,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           c2[e] = (Jb <= 1) ? ex2(Rnext[e] - GeJ[e]) : 0.f;
           c3[e] = (Jb == 0) ? ex2(refg[2 * kD + j0 + e] - GeJ[e]) : 0.f;
         }
+        uint4 qraw[4], kraw[4];
+        float rqv[4], rkv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int r = r0 + i;
-          const bool valid = r < n;
+          qraw[i] = *reinterpret_cast<const uint4*>(sQ + sw128_offset(64, r0 + i, j0));
+          kraw[i] = *reinterpret_cast<const uint4*>(sK + sw128_offset(64, r0 + i, j0));
           float qv[8], kv[8];
-          unpack8(*reinterpret_cast<const uint4*>(sQ + sw128_offset(64, r, j0)), qv);
-          unpack8(*reinterpret_cast<const uint4*>(sK + sw128_offset(64, r, j0)), kv);
+          unpack8(qraw[i], qv);
+          unpack8(kraw[i], kv);
           float ssq = 0.f, ssk = 0.f;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             ssq = fmaf(qv[e], qv[e], ssq);
             ssk = fmaf(kv[e], kv[e], ssk);
           }
+          rqv[i] = ssq;
+          rkv[i] = ssk;
+        }
 #pragma unroll
-          for (int o = 1; o < 16; o <<= 1) {
-            ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
-            ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
+        for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            rqv[i] += __shfl_xor_sync(0xffffffffu, rqv[i], o);
+            rkv[i] += __shfl_xor_sync(0xffffffffu, rkv[i], o);
           }
-          const float rq = rsqrtf(ssq + 1e-6f) * p.scale;
-          const float rk = rsqrtf(ssk + 1e-6f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = r0 + i;
+          const bool valid = r < n;
+          float qv[8], kv[8];
+          unpack8(qraw[i], qv);
+          unpack8(kraw[i], kv);
+          const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
+          const float rk = rsqrtf(rkv[i] + 1e-6f);
           float ka[8], qa[8], kt[8], qt[8], kh[8], khl[8], b0[8], b1[8], b2[8], b3[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -391,23 +479,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(sK + sw128_offset(64, r, j0)) = pack8(kh);
           khlo[i] = pack8(khl);
           *reinterpret_cast<uint4*>(sG + sw128_offset(64, r, j0)) = pack8(kt);
-          *reinterpret_cast<uint4*>(sm + SM_BT + btoff(Jb) + sw128_offset(16 * (Jb + 1), r, j0)) =
+          *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb) + r, j0)) =
               pack8(b0);
           if (Jb + 1 <= 3)
-            *reinterpret_cast<uint4*>(sm + SM_BT + btoff(Jb + 1) +
-                                      sw128_offset(16 * (Jb + 2), r, j0)) = pack8(b1);
+            *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 1) + r, j0)) = pack8(b1);
           if (Jb + 2 <= 3)
-            *reinterpret_cast<uint4*>(sm + SM_BT + btoff(Jb + 2) +
-                                      sw128_offset(16 * (Jb + 3), r, j0)) = pack8(b2);
+            *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 2) + r, j0)) = pack8(b2);
           if (Jb + 3 <= 3)
-            *reinterpret_cast<uint4*>(sm + SM_BT + btoff(Jb + 3) +
-                                      sw128_offset(16 * (Jb + 4), r, j0)) = pack8(b3);
+            *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 3) + r, j0)) = pack8(b3);
           if (!valid) *reinterpret_cast<uint4*>(sV + sw128_offset(64, r, j0)) = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
+      KDA_TS(2);
       if (*abort_flag) {
         aborted = true;
         break;
@@ -416,114 +502,136 @@ __global__ void __launch_bounds__(kThreads, 1)
       // =================== phase 2: intra MMAs ===================
       if (tid == 0) {
         tc_fence_after();
+        // D[:, 0:160] = Aop [B^(0); B^(1); B^(2); B^(3)]^T in one N=160 MMA chain: D_I = cols dcol(I)..
+        const uint32_t idesc = idesc_bf16(128, BT_ROWS, 0, 0);
 #pragma unroll
-        for (int I = 0; I < 4; ++I) {
-          const uint32_t N = 16u * (I + 1);
-          const uint32_t idesc = idesc_bf16(128, N, 0, 0);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = smem_desc(sbase + SM_AOP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd =
-                smem_desc(sbase + SM_BT + btoff(I) + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-            mma_ss(tbase + TC_D + dcol(I), ad, bd, idesc, kk > 0);
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = smem_desc(sbase + SM_AOP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc(sbase + SM_BT + (kk >> 2) * (BT_ROWS * 128) + (kk & 3) * 32, 16, 1024);
+          mma_ss(tbase + TC_D, ad, bd, idesc, kk > 0);
         }
         mma_commit(bar_mma);
       }
       wait_mma();
+      KDA_TS(3);
       tc_fence_after();
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         *reinterpret_cast<uint4*>(sm + SM_KLO + sw128_offset(64, r0 + i, j0)) = khlo[i];
 
       // =================== phase 3: T, Aqk, solve ===================
-      float* Ts = reinterpret_cast<float*>(sm + SM_BT);  // [64][65]
-      float* Xs = Ts + 64 * 65;                           // [64][65]
-      float* Ms = Xs + 64 * 65;                           // [3][16][17]
-      if (warp < 4) {
-        const int r = (warp & 1) * 32 + lane;  // row within the chunk
-        const int I = r >> 4;
-        const bool krow = warp < 2;
+      // fp32 scratch in the B-tile region (free once the intra MMA has completed)
+      constexpr int TP = 68, YP = 36;                       // row pitches (floats)
+      float* Ts = reinterpret_cast<float*>(sm + SM_BT);   // T = stril(diag(beta) K~ K-^T) [64][TP]
+      float* Xs = Ts + 64 * TP;                           // X = (I + T)^-1            [64][TP]
+      float* Ys = Xs + 64 * TP;                           // block products            [32][YP]
+      {
+        // warp w: lane quarter q = w & 3 (q < 2: k rows -> T; q >= 2: q rows -> Aqk), row block
+        // blk = 2 (q & 1) + (w >> 2); one batched TMEM load of D_blk, then the 16 lanes of that
+        // block write their rows.  X is cleared alongside.
+        const int q4 = warp & 3;
+        const int r = (q4 & 1) * 32 + lane;
+        const int blk = 2 * (q4 & 1) + (warp >> 2);
+        const bool krow = q4 < 2;
         const float br = krow ? beta_s[r] : 0.f;
-#pragma unroll
-        for (int bi = 0; bi < 2; ++bi) {
-          const int blk = (warp & 1) * 2 + bi;
-          for (int ch = 0; ch <= blk; ++ch) {
-            uint32_t v[16];
-            tmem_ld16(tbase + wlane + TC_D + dcol(blk) + 16 * ch, v);
-            tmem_wait_ld();
-            if (I == blk) {
-              if (krow) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  const int s = 16 * ch + e;
-                  Ts[r * 65 + s] = (s < r) ? br * __uint_as_float(v[e]) : 0.f;
-                }
-              } else {
-                float f[8];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) {
-                    const int s = 16 * ch + 8 * hh + e;
-                    f[e] = (s <= r) ? __uint_as_float(v[8 * hh + e]) : 0.f;
-                  }
-                  *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch + 8 * hh)) = pack8(f);
-                }
-              }
-            }
-          }
+        const uint32_t ta = tbase + wlane + TC_D;
+        switch (blk) {
+          case 0: extract_block<0>(ta, r, krow, br, Ts, sm + SM_AQK); break;
+          case 1: extract_block<1>(ta, r, krow, br, Ts, sm + SM_AQK); break;
+          case 2: extract_block<2>(ta, r, krow, br, Ts, sm + SM_AQK); break;
+          default: extract_block<3>(ta, r, krow, br, Ts, sm + SM_AQK); break;
         }
-        // columns past this row block are zero
-        for (int s = 16 * (I + 1); s < 64; s += 8) {
-          if (krow) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) Ts[r * 65 + s + e] = 0.f;
-          } else {
-            *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, s)) = make_uint4(0, 0, 0, 0);
-          }
-        }
+        for (int e = tid; e < 64 * TP / 4; e += kThreads)
+          reinterpret_cast<float4*>(Xs)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       __syncthreads();
-      // diagonal 16x16 blocks: X_II = (I + T_II)^-1, one column per thread
+      KDA_TS(13);
+      // level 1: X_II = (I + T_II)^-1 for the four 16x16 diagonal blocks, one column per thread
       if (tid < 64) {
         const int I = tid >> 4, cc = tid & 15, base = 16 * I;
         float x[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) x[k] = (k == cc) ? 1.f : 0.f;
+        // outer-product order: once x[k] is final, update every later row (independent FMAs)
 #pragma unroll
-        for (int rr = 1; rr < 16; ++rr) {
-          float acc = x[rr];
+        for (int k = 0; k < 15; ++k) {
 #pragma unroll
-          for (int k = 0; k < rr; ++k) acc = fmaf(-Ts[(base + rr) * 65 + base + k], x[k], acc);
-          x[rr] = acc;
+          for (int rr = k + 1; rr < 16; ++rr) x[rr] = fmaf(-Ts[(base + rr) * TP + base + k], x[k], x[rr]);
         }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) Xs[(base + k) * 65 + base + cc] = x[k];
+        for (int k = 0; k < 16; ++k) Xs[(base + k) * TP + base + cc] = x[k];
       }
       __syncthreads();
-      // off-diagonal blocks by distance d: X_IJ = -X_II sum_{K=J}^{I-1} T_IK X_KJ
-      for (int d = 1; d <= 3; ++d) {
-        const int nblk = 4 - d;
-        for (int e = tid; e < nblk * 256; e += kThreads) {
-          const int pI = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-          const int I = d + pI, J = I - d;
-          float acc = 0.f;
-          for (int k = 16 * J + cc; k < 16 * I; ++k)
-            acc = fmaf(Ts[(16 * I + rr) * 65 + k], Xs[k * 65 + 16 * J + cc], acc);
-          Ms[(pI * 16 + rr) * 17 + cc] = acc;
+      KDA_TS(14);
+      // level 2: X_{I,I-1} = -X_II T_{I,I-1} X_{I-1,I-1} for I = 1, 3 (two 16x16 merges)
+      {
+        const int pI = tid >> 7, rr = (tid >> 3) & 15, c0 = (tid & 7) * 2;
+        const int I = 2 * pI + 1, J = I - 1;
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float t = Ts[(16 * I + rr) * TP + 16 * J + k];
+          const float2 xv = *reinterpret_cast<const float2*>(Xs + (16 * J + k) * TP + 16 * J + c0);
+          y0 = fmaf(t, xv.x, y0);
+          y1 = fmaf(t, xv.y, y1);
         }
+        *reinterpret_cast<float2*>(Ys + (16 * pI + rr) * YP + c0) = make_float2(y0, y1);
         __syncthreads();
-        for (int e = tid; e < nblk * 256; e += kThreads) {
-          const int pI = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-          const int I = d + pI, J = I - d;
-          float acc = 0.f;
-          for (int k = 0; k <= rr; ++k)
-            acc = fmaf(Xs[(16 * I + rr) * 65 + 16 * I + k], Ms[(pI * 16 + k) * 17 + cc], acc);
-          Xs[(16 * I + rr) * 65 + 16 * J + cc] = -acc;
+        float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float xx = Xs[(16 * I + rr) * TP + 16 * I + k];
+          const float2 yv = *reinterpret_cast<const float2*>(Ys + (16 * pI + k) * YP + c0);
+          z0 = fmaf(xx, yv.x, z0);
+          z1 = fmaf(xx, yv.y, z1);
         }
-        __syncthreads();
+        *reinterpret_cast<float2*>(Xs + (16 * I + rr) * TP + 16 * J + c0) = make_float2(-z0, -z1);
       }
+      __syncthreads();
+      KDA_TS(15);
+      // level 3: X_(32:64, 0:32) = -X_(32:64, 32:64) T_(32:64, 0:32) X_(0:32, 0:32) (32x32 merge);
+      // each thread owns a 2x2 output tile (rows 2 tr, 2 tr + 1; columns 2 tc, 2 tc + 1)
+      {
+        const int tr = tid >> 4, tc = tid & 15;
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 4) {
+          const float4 ta = *reinterpret_cast<const float4*>(Ts + (32 + 2 * tr) * TP + k0);
+          const float4 tb = *reinterpret_cast<const float4*>(Ts + (33 + 2 * tr) * TP + k0);
+          const float tav[4] = {ta.x, ta.y, ta.z, ta.w}, tbv[4] = {tb.x, tb.y, tb.z, tb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 xv = *reinterpret_cast<const float2*>(Xs + (k0 + e) * TP + 2 * tc);
+            y00 = fmaf(tav[e], xv.x, y00);
+            y01 = fmaf(tav[e], xv.y, y01);
+            y10 = fmaf(tbv[e], xv.x, y10);
+            y11 = fmaf(tbv[e], xv.y, y11);
+          }
+        }
+        *reinterpret_cast<float2*>(Ys + (2 * tr) * YP + 2 * tc) = make_float2(y00, y01);
+        *reinterpret_cast<float2*>(Ys + (2 * tr + 1) * YP + 2 * tc) = make_float2(y10, y11);
+        __syncthreads();
+        float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 4) {
+          const float4 xa = *reinterpret_cast<const float4*>(Xs + (32 + 2 * tr) * TP + 32 + k0);
+          const float4 xb = *reinterpret_cast<const float4*>(Xs + (33 + 2 * tr) * TP + 32 + k0);
+          const float xav[4] = {xa.x, xa.y, xa.z, xa.w}, xbv[4] = {xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 yv = *reinterpret_cast<const float2*>(Ys + (k0 + e) * YP + 2 * tc);
+            z00 = fmaf(xav[e], yv.x, z00);
+            z01 = fmaf(xav[e], yv.y, z01);
+            z10 = fmaf(xbv[e], yv.x, z10);
+            z11 = fmaf(xbv[e], yv.y, z11);
+          }
+        }
+        *reinterpret_cast<float2*>(Xs + (32 + 2 * tr) * TP + 2 * tc) = make_float2(-z00, -z01);
+        *reinterpret_cast<float2*>(Xs + (33 + 2 * tr) * TP + 2 * tc) = make_float2(-z10, -z11);
+      }
+      __syncthreads();
+      KDA_TS(16);
       // Xsol = X diag(beta) -> bf16 hi and lo parts, K-major [r][s]
       {
         const int r = tid >> 2, s0 = (tid & 3) * 16;
@@ -533,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int s = s0 + 8 * hh + e;
-            f[e] = (s <= r) ? Xs[r * 65 + s] * beta_s[s] : 0.f;
+            f[e] = (s <= r) ? Xs[r * TP + s] * beta_s[s] : 0.f;
             fl[e] = f[e] - bf16_round(f[e]);
           }
           *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(64, r, s0 + 8 * hh)) = pack8(f);
@@ -543,44 +651,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
+      KDA_TS(4);
 
       // =================== phase 4: W^T and U^T ===================
       if (tid == 0) {
         tc_fence_after();
         const uint32_t idesc = idesc_bf16(128, 64, 1, 0);
+        // W first (its epilogue waits on this commit), then U (consumed in order by phase 5)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024);
-          const uint64_t bl = smem_desc(sbase + SM_XWLO + kk * 32, 16, 1024);
           const uint64_t aw = smem_desc(aG + kk * 2048, 8192, 1024);
+          mma_ss(tbase + TC_D, aw, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc, kk > 0);
+          mma_ss(tbase + TC_D, aw, smem_desc(sbase + SM_XWLO + kk * 32, 16, 1024), idesc, 1);
+        }
+        if (!dbg) mma_commit(bar_mma);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
           const uint64_t av = smem_desc(aV + kk * 2048, 8192, 1024);
-          mma_ss(tbase + TC_D, aw, bd, idesc, kk > 0);
-          mma_ss(tbase + TC_D, aw, bl, idesc, 1);
-          mma_ss(tbase + TC_DELTA, av, bd, idesc, kk > 0);
-          mma_ss(tbase + TC_DELTA, av, bl, idesc, 1);
+          mma_ss(tbase + TC_DELTA, av, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc, kk > 0);
+          mma_ss(tbase + TC_DELTA, av, smem_desc(sbase + SM_XWLO + kk * 32, 16, 1024), idesc, 1);
         }
-        mma_commit(bar_mma);
+        if (dbg) mma_commit(bar_mma);  // the debug dump reads U too
       }
-      wait_mma();
-      tc_fence_after();
       {
-        const int j = wq + lane;
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t v[16];
-          tmem_ld16(tbase + wlane + TC_D + wg * 32 + 16 * ch, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int r = wg * 32 + 16 * ch + e;
-            const float wv = -__uint_as_float(v[e]);
-            const __nv_bfloat16 whi = __float2bfloat16_rn(wv);
-            *reinterpret_cast<__nv_bfloat16*>(sG + sw128_offset(64, r, j)) = whi;
-            *reinterpret_cast<__nv_bfloat16*>(sm + SM_XWLO + sw128_offset(64, r, j)) =
-                __float2bfloat16_rn(wv - __bfloat162float(whi));
-          }
-        }
-        // lo part of the bf16 state operand: S - bf16(S) for this warpgroup's 64 columns
+        // lo part of the bf16 state operand, S - bf16(S), built while the W/U MMAs run (they
+        // touch neither TC_S nor TC_SLO)
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t v0[16], v1[16], pk[16];
@@ -598,6 +693,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(tbase + wlane + TC_SLO + col / 2, pk);
         }
         tmem_wait_st();
+      }
+      wait_mma();
+      KDA_TS(5);
+      tc_fence_after();
+      {
+        // W^T row j (tokens r = 32 wg .. 32 wg + 31) -> -W^T stored MN-major: tile [j][r], one atom
+        const int j = wq + lane;
+        uint32_t vw[2][16];
+        tmem_ld16(tbase + wlane + TC_D + wg * 32, vw[0]);
+        tmem_ld16(tbase + wlane + TC_D + wg * 32 + 16, vw[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const uint32_t* v = vw[ch];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float hi[8], lo[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float wv = -__uint_as_float(v[8 * hh + e]);
+              hi[e] = wv;
+              lo[e] = wv - bf16_round(wv);
+            }
+            const int rc = wg * 32 + 16 * ch + 8 * hh;  // first token of this 8-wide chunk
+            *reinterpret_cast<uint4*>(sG + sw128_offset(128, j, rc)) = pack8(hi);
+            *reinterpret_cast<uint4*>(sm + SM_XWLO + sw128_offset(128, j, rc)) = pack8(lo);
+          }
+        }
       }
       if (dbg) {  // per-chunk intermediates in the two-kernel workspace layout (fp32)
         float* dc = dbg + (size_t)(coff + c) * (kWsChunkBytes / 4);
@@ -627,67 +750,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
+      KDA_TS(6);
 
       // =================== phase 5: Delta^T = U^T - S0 W^T,  O^T = S0 Q~^T ===================
       if (tid == 0) {
         tc_fence_after();
         const uint32_t idesc = idesc_bf16(128, 64, 0, 0);
+        const uint32_t idesc_w = idesc_bf16(128, 64, 0, 1);  // -W^T tiles are MN-major [j][r]
+        // Delta first (phase 6 waits on this commit); O^T = S0 Q~^T after it, covered by the
+        // commit of phase 7
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bw = smem_desc(aG + kk * 2048, 16384, 1024);
+          mma_ts(tbase + TC_DELTA, tbase + TC_S0 + kk * 8, bw, idesc_w, 1);
+          mma_ts(tbase + TC_DELTA, tbase + TC_SLO + kk * 8, bw, idesc_w, 1);
+          mma_ts(tbase + TC_DELTA, tbase + TC_S0 + kk * 8,
+                 smem_desc(sbase + SM_XWLO + kk * 2048, 16384, 1024), idesc_w, 1);
+        }
+        mma_commit(bar_mma);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-          const uint64_t bw = smem_desc(aG + koff, 16, 1024);
-          mma_ts(tbase + TC_DELTA, tbase + TC_S0 + kk * 8, bw, idesc, 1);
-          mma_ts(tbase + TC_DELTA, tbase + TC_SLO + kk * 8, bw, idesc, 1);
-          mma_ts(tbase + TC_DELTA, tbase + TC_S0 + kk * 8,
-                 smem_desc(sbase + SM_XWLO + koff, 16, 1024), idesc, 1);
           mma_ts(tbase + TC_O, tbase + TC_S0 + kk * 8, smem_desc(aQ + koff, 16, 1024), idesc, kk > 0);
         }
-        mma_commit(bar_mma);
+      }
+      if (wg == 1) {
+        // S <- S Diag(2^G_last) while the Delta/O MMAs run (they read the bf16 copies, not TC_S)
+#pragma unroll
+        for (int ch = 0; ch < 8; ch += 2) {
+          uint32_t v[16], w2[16];
+          tmem_ld16(tbase + wlane + TC_S + 16 * ch, v);
+          tmem_ld16(tbase + wlane + TC_S + 16 * ch + 16, w2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            v[e] = __float_as_uint(__uint_as_float(v[e]) * gcs[16 * ch + e]);
+            w2[e] = __float_as_uint(__uint_as_float(w2[e]) * gcs[16 * ch + 16 + e]);
+          }
+          tmem_st16(tbase + wlane + TC_S + 16 * ch, v);
+          tmem_st16(tbase + wlane + TC_S + 16 * ch + 16, w2);
+        }
+        tmem_wait_st();
       }
       wait_mma();
+      KDA_TS(7);
       tc_fence_after();
 
-      // =================== phase 6: Delta^T -> bf16;  S <- S Diag(2^G_last) ===================
-      if (wg == 0) {
-        uint32_t pk[32], pl[32];
+      // =================== phase 6: Delta^T -> bf16 hi and lo ===================
+      {
+        // warpgroup wg converts tokens 32 wg .. 32 wg + 31 (one batched load of 32 columns)
+        uint32_t v0[16], v1[16], hi[16], lo[16];
+        tmem_ld16(tbase + wlane + TC_DELTA + 32 * wg, v0);
+        tmem_ld16(tbase + wlane + TC_DELTA + 32 * wg + 16, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t v[16];
-          tmem_ld16(tbase + wlane + TC_DELTA + 16 * ch, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float d0 = __uint_as_float(v[2 * e]), d1 = __uint_as_float(v[2 * e + 1]);
-            pk[8 * ch + e] = pack_bf16(d0, d1);
-            pl[8 * ch + e] = pack_bf16(d0 - bf16_round(d0), d1 - bf16_round(d1));
-          }
+        for (int e = 0; e < 8; ++e) {
+          const float d0 = __uint_as_float(v0[2 * e]), d1 = __uint_as_float(v0[2 * e + 1]);
+          const float d2 = __uint_as_float(v1[2 * e]), d3 = __uint_as_float(v1[2 * e + 1]);
+          hi[e] = pack_bf16(d0, d1);
+          hi[8 + e] = pack_bf16(d2, d3);
+          lo[e] = pack_bf16(d0 - bf16_round(d0), d1 - bf16_round(d1));
+          lo[8 + e] = pack_bf16(d2 - bf16_round(d2), d3 - bf16_round(d3));
         }
-        uint32_t a[16], bq[16], la[16], lb[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          a[e] = pk[e];
-          bq[e] = pk[16 + e];
-          la[e] = pl[e];
-          lb[e] = pl[16 + e];
-        }
-        tmem_st16(tbase + wlane + TC_DB, a);
-        tmem_st16(tbase + wlane + TC_DB + 16, bq);
-        tmem_st16(tbase + wlane + TC_DLO, la);
-        tmem_st16(tbase + wlane + TC_DLO + 16, lb);
-      } else {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t v[16];
-          tmem_ld16(tbase + wlane + TC_S + 16 * ch, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * gcs[16 * ch + e]);
-          tmem_st16(tbase + wlane + TC_S + 16 * ch, v);
-        }
+        tmem_st16(tbase + wlane + TC_DB + 16 * wg, hi);
+        tmem_st16(tbase + wlane + TC_DLO + 16 * wg, lo);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncthreads();
+      KDA_TS(8);
 
       // =================== phase 7: S += Delta^T K^,  O^T += Delta^T Aqk^T ===================
       if (tid == 0) {
@@ -707,28 +838,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_mma);
       }
       wait_mma();
+      KDA_TS(9);
       if (tid == 0 && !*abort_flag) {
         fence_proxy_async_smem();
         produce();  // the slot of this chunk is free: bring in the chunk after next
       }
+      KDA_TS(17);
       tc_fence_after();
 
       // =================== phase 8: out rows;  S -> bf16 operand (and final_state) ===================
       {
         const int i = wq + lane;
-        const int64_t ostride = (p.layout == KDA_LAYOUT_BNSD) ? kD : (int64_t)p.Nv * kD;
-        __nv_bfloat16* orow = p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t0) + i;
+        uint32_t vo[2][16];
+        tmem_ld16(tbase + wlane + TC_O + wg * 32, vo[0]);
+        tmem_ld16(tbase + wlane + TC_O + wg * 32 + 16, vo[1]);
+        tmem_wait_ld();
+        if (n == kChunk) {
+          // full chunk: out tile [t][i] (128B-swizzled, as the out tensor map expects) in the free
+          // Aop region, then two TMA stores issued below
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t v[16];
-          tmem_ld16(tbase + wlane + TC_O + wg * 32 + 16 * ch, v);
-          tmem_wait_ld();
+          for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int t = wg * 32 + 16 * ch + e;
-            if (t < n) orow[t * ostride] = __float2bfloat16_rn(__uint_as_float(v[e]));
-          }
+            for (int e = 0; e < 16; ++e) {
+              const int t = wg * 32 + 16 * ch + e;
+              *reinterpret_cast<__nv_bfloat16*>(sm + SM_OSTG + sw128_offset(64, t, i)) =
+                  __float2bfloat16_rn(__uint_as_float(vo[ch][e]));
+            }
+        } else {
+          // the sequence's last, partial chunk: plain stores of the valid rows
+          const int64_t ostride = (p.layout == KDA_LAYOUT_BNSD) ? kD : (int64_t)p.Nv * kD;
+          __nv_bfloat16* orow = p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t0) + i;
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int t = wg * 32 + 16 * ch + e;
+              if (t < n) orow[t * ostride] = __float2bfloat16_rn(__uint_as_float(vo[ch][e]));
+            }
         }
+        KDA_TS(18);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t v0[16], v1[16], pk[16];
@@ -757,8 +905,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       }
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
+      KDA_TS(10);
+      if (tid == 0 && n == kChunk) {
+        int oc1, oc2;
+        if (p.layout == KDA_LAYOUT_BNSD) {
+          oc1 = t0;
+          oc2 = b * p.Nv + h;
+        } else {
+          oc1 = h;
+          oc2 = (p.layout == KDA_LAYOUT_BSND ? b * p.S : tok0) + t0;
+        }
+        tma_store_3d(&maps.o, sbase + SM_OSTG, 0, oc1, oc2);
+        tma_store_3d(&maps.o, sbase + SM_OSTG + 8192, 64, oc1, oc2);
+        tma_store_commit();
+      }
       if (*abort_flag) {
         aborted = true;
         break;
@@ -774,8 +937,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // drain: loads still in flight must land before this CTA's shared memory goes away
+  // drain: loads still in flight must land, and stores complete, before this CTA exits
   if (tid == 0) {
+    tma_store_wait_all();
     while (gidx < issued) {
       if (!mbar_wait_bounded(sbase + SM_BAR + 8u * (gidx & 1), (gidx >> 1) & 1u, kWaitLimit)) {
         atomicExch(p.status, DS_TIMEOUT);
@@ -827,7 +991,8 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
   if (!make_map(&m.q, p.q, p.layout, p.B, p.Nqk, p.S) ||
       !make_map(&m.k, p.k, p.layout, p.B, p.Nqk, p.S) ||
       !make_map(&m.v, p.v, p.layout, p.B, p.Nv, p.S) ||
-      !make_map(&m.g, p.g, p.layout, p.B, p.Nv, p.S))
+      !make_map(&m.g, p.g, p.layout, p.B, p.Nv, p.S) ||
+      !make_map(&m.o, p.out, p.layout, p.B, p.Nv, p.S))
     return cudaErrorInvalidValue;
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   kda_fused_kernel<<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);

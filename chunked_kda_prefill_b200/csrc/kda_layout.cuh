@@ -27,6 +27,7 @@ struct Params {
   int32_t* status;
   __nv_bfloat16* out;
   float* Sf;
+  unsigned long long* tprof;  // optional: CTA 0 records clock64() at phase boundaries
 };
 
 // Element offset of the D-vector of (sequence b, head hx of NX heads, token t of the sequence).
@@ -71,7 +72,8 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
                           const void* v, const void* g, const void* beta, float scale,
                           const float* initial_state, const float* A_log, const float* dt_bias,
                           float lower_bound, void* workspace, size_t workspace_bytes, void* out,
-                          float* final_state, cudaStream_t stream, float* dbg);
+                          float* final_state, cudaStream_t stream, float* dbg,
+                          unsigned long long* tprof = nullptr);
 
 // Workspace bytes of the two-kernel path for a validated plan.
 size_t simt_workspace_bytes(const int32_t* plan);

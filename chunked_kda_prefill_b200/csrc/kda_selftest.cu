@@ -25,6 +25,8 @@ enum : int {
   ST_TS_K = 3,     // A from TMEM, B K-major
   ST_TMA = 4,      // TMA load of a 64x128 box pair, raw shared-memory bytes out
   ST_TS_MN = 5,    // A from TMEM, B MN-major
+  ST_TF32_SS = 6,  // kind::tf32, A K-major fp32, B K-major fp32 (shared memory)
+  ST_TF32_TS = 7,  // kind::tf32, A fp32 from TMEM, B K-major fp32
 };
 
 constexpr uint32_t kWaitLimit = 1u << 24;
@@ -56,7 +58,57 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tbase = *tslot;
 
-  if (variant == ST_TMA) {
+  if (variant == ST_TF32_SS || variant == ST_TF32_TS) {
+    // fp32 operands (tf32 MMA): A [128][K] (fp32, passed as A), B [N][K] (fp32), both K-major
+    const float* Af = reinterpret_cast<const float*>(A);
+    const float* Bf = reinterpret_cast<const float*>(B);
+    const bool a_tmem = (variant != ST_TF32_SS);
+    if (!a_tmem) {
+      for (int e = tid; e < 128 * K; e += 128) {
+        const int m = e / K, k = e % K;
+        *reinterpret_cast<float*>(sA + sw128_offset_f32(128, m, k)) = Af[e];
+      }
+    } else {
+      const int m = tid;
+      for (int c0 = 0; c0 < K; c0 += 16) {
+        uint32_t r[16];
+        for (int c = 0; c < 16; ++c) r[c] = __float_as_uint(Af[m * K + c0 + c]);
+        tmem_st16(tbase + ((uint32_t)(warp * 32) << 16) + 256 + c0, r);
+      }
+      tmem_wait_st();
+    }
+    for (int e = tid; e < N * K; e += 128) {
+      const int n = e / K, k = e % K;
+      *reinterpret_cast<float*>(sB + sw128_offset_f32(N, n, k)) = Bf[e];
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_tf32(128, N, 0u, 0u);
+      for (int kk = 0; kk < K / 8; ++kk) {
+        const uint64_t bd =
+            smem_desc(smem_u32(sB) + (kk / 4) * (N * 128) + (kk % 4) * 32, 16, 1024);
+        if (a_tmem) {
+          mma_ts_tf32(tbase, tbase + 256 + kk * 8, bd, idesc, kk > 0);
+        } else {
+          const uint64_t ad =
+              smem_desc(smem_u32(sA) + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
+          mma_ss_tf32(tbase, ad, bd, idesc, kk > 0);
+        }
+      }
+      mma_commit(bar_a);
+    }
+    if (!mbar_wait_bounded(bar_a, 0, kWaitLimit) && tid == 0) atomicExch(err, 2);
+    tc_fence_after();
+    for (int c0 = 0; c0 < N; c0 += 16) {
+      uint32_t r[16];
+      tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + c0, r);
+      tmem_wait_ld();
+      for (int c = 0; c < 16; ++c) D[tid * N + c0 + c] = __uint_as_float(r[c]);
+    }
+  } else if (variant == ST_TMA) {
     if (tid == 0) {
       mbar_arrive_expect_tx(bar_a, 16384);
       tma_load_3d(smem_u32(sA), &tmap, bar_a, 0, row0, 0);
@@ -144,10 +196,10 @@ extern "C" __attribute__((visibility("default"))) int kda_selftest(
     int variant, const void* A, const void* B, float* D, int N, int K, void* raw,
     const void* tma_src, int tma_rows, int row0, int* err_dev, void* stream) {
   using namespace kda;
-  if (variant < 0 || variant > 5) return 1;
-  if (variant != ST_TMA && (!A || !B || !D || (K != 64 && K != 128) || N < 16 || N > 128 ||
-                            N % 16 != 0))
-    return 1;
+  if (variant < 0 || variant > ST_TF32_TS) return 1;
+  if (variant != ST_TMA && (!A || !B || !D || N < 16 || N > 128 || N % 16 != 0)) return 1;
+  if (variant != ST_TMA && variant < ST_TF32_SS && K != 64 && K != 128) return 1;
+  if (variant >= ST_TF32_SS && K != 32 && K != 64) return 1;
   if ((variant == ST_SS_KMN || variant == ST_TS_MN) && N != 64 && N != 128) return 1;
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));

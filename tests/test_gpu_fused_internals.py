@@ -30,7 +30,7 @@ def _bind(L):
     L.kda_forward_simt.argtypes = [sh, P, vp, sz, vp, vp, vp, vp, vp, f, vp, vp, vp, f, vp, sz,
                                    vp, vp, vp]
     L.kda_forward_debug.argtypes = [sh, P, vp, sz, vp, vp, vp, vp, vp, f, vp, vp, vp, f, vp, sz,
-                                    vp, vp, vp, vp]
+                                    vp, vp, vp, vp, vp]
     L.kda_simt_workspace_size.argtypes = [P, sz, ctypes.POINTER(sz)]
     for n in ("kda_forward_simt", "kda_forward_debug", "kda_simt_workspace_size"):
         getattr(L, n).restype = ctypes.c_int
@@ -64,7 +64,7 @@ def _run_both(w):
             torch.cuda.synchronize()
             simt_ws = ws[256:].view(torch.float32).clone()
         else:
-            assert L.kda_forward_debug(*args(out, fs), dump.data_ptr() + 256, s) == 0
+            assert L.kda_forward_debug(*args(out, fs), dump.data_ptr() + 256, None, s) == 0
             torch.cuda.synchronize()
         kda.device_status(ws)
         outs[name] = (out.float().cpu().numpy(), fs.cpu().numpy())

@@ -70,3 +70,26 @@ def test_tma_swizzle_matches_hand_layout(cuda_ok):
     for r in range(64):
         for c in range(128):
             assert raw_h[_sw128(64, r, c) // 2] == s[row0 + r, c], (r, c)
+
+
+def _tf32(x):
+    """Round-toward-zero to tf32 (keep 10 mantissa bits) so the MMA sees exactly these values."""
+    u = x.contiguous().view(torch.int32) & ~0x1FFF
+    return u.view(torch.float32)
+
+
+@pytest.mark.parametrize("variant,N,K", [(6, 64, 64), (6, 128, 32), (7, 64, 64), (7, 128, 32)])
+def test_tf32_mma_plumbing(variant, N, K, cuda_ok):
+    f = _lib()
+    g = torch.Generator().manual_seed(300 + variant * 11 + N + K)
+    A = _tf32(torch.randn(128, K, generator=g))
+    B = _tf32(torch.randn(N, K, generator=g))
+    a_d, b_d = A.cuda(), B.cuda()
+    D = torch.full((128, N), float("nan"), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = f(variant, a_d.data_ptr(), b_d.data_ptr(), D.data_ptr(), N, K, None, None, 0, 0,
+           err.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    ref = A.double() @ B.double().t()
+    got = D.cpu().double()
+    assert torch.allclose(got, ref, rtol=1e-5, atol=1e-4), (got - ref).abs().max()
