@@ -1,6 +1,6 @@
-// kda_fused.cu -- fused chunked KDA prefill for sm_100a: one persistent CTA per (sequence, value
-// head) unit at a time, tcgen05 tensor cores for every contraction, the 128x128 fp32 state kept in
-// TMEM for the whole sequence.
+// kda_fused.cu -- fused chunked KDA prefill for sm_100a: one persistent CTA of 16 warps per SM,
+// one (sequence, value head) unit at a time, tcgen05 tensor cores for every contraction, the
+// 128x128 fp32 state kept in TMEM for the whole sequence.
 //
 // Per 64-token chunk (the chunk equations of the FlashKDA README, 功能说明), eight phases:
 //   1 prologue (CUDA cores): gate activation g = lb*sigmoid(e^A_log*(g_raw+dt_bias)) in log2
@@ -9,18 +9,22 @@
 //     no factor overflows (the sub-chunk reference point b_gn of vLLM PR 43195's excerpt):
 //       Aop = [k^ 2^(G-ref_I) ; scale q^ 2^(G-ref_I)],  B^(I) rows = k^ 2^(ref_I - G)  (s < 16(I+1)),
 //       K~ = k^ 2^G, Q~ = scale q^ 2^G, K^ = k^ 2^(G_last - G)   (written over the raw q/k/g tiles)
-//   2 MMA  D_I = Aop B^(I)^T, I = 0..3 (M=128, N=16(I+1), K=128): rows 0-63 give
+//   2 MMA  D_I = Aop B^(I)^T, I = 0..3 (M=128, N=160 for all four blocks, K=128): rows 0-63 give
 //     T = stril(diag(beta) K~ K-^T), rows 64-127 give Aqk = tril(Q~ K-^T)
-//   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 16x16 diagonal blocks and off-diagonal updates;
-//     Xsol = X diag(beta) -> bf16
-//   4 MMA  W^T = K~^T Xsol^T and U^T = V^T Xsol^T (M=128, N=64, K=64); W -> -W bf16
-//   5 MMA  Delta^T = U^T + S0 (-W)^T and O^T = S0 Q~^T (A = bf16 state read from TMEM)
-//   6 Delta^T -> bf16 in TMEM;  S <- S Diag(2^G_last)
-//   7 MMA  S += Delta^T K^,  O^T += Delta^T Aqk^T   (then TMA for the chunk after next)
-//   8 O^T -> bf16 out;  S -> bf16 state operand (and fp32 final_state after the last chunk)
-// Operands that feed the state recurrence (Xsol, W, S0, Delta, K^) are split into bf16 hi + lo
+//   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 16x16 diagonal blocks and two merge levels;
+//     Xsol = X diag(beta) -> bf16 hi and lo parts stacked as one 128-row operand
+//   4 MMA  W^T = K~^T [Xsol_hi; Xsol_lo]^T (one N=128 chain), U^T = V^T Xsol^T; S <- S Diag(2^G_last)
+//     meanwhile.  Then -W -> bf16 hi and lo, stored token-major over the K~ and V tiles
+//   5 MMA  [O^T | Da | Db] = S_hi [Q~ | -W_hi | -W_lo]^T (N=192) and [O^T | Da] += S_lo [Q~ | -W_hi]^T
+//     (A operand = bf16 state in TMEM); Delta^T = U^T + Da + Db
+//   6 Delta^T -> bf16 hi and lo in TMEM
+//   7 MMA  S += Delta^T K^ (hi/lo),  O^T += Delta^T Aqk^T   (then TMA for the chunk after next)
+//   8 O^T -> bf16 out (TMA store);  S -> bf16 hi and lo state operand (fp32 final_state at the end)
+// Operands that feed the state recurrence (Xsol, W, S, Delta, K^) are split into bf16 hi + lo
 // parts and multiplied as hi*hi + lo*hi + hi*lo, so the state path keeps ~16 significant bits
 // instead of bf16's 8: without that, rounding errors pile up when the gate does not decay.
+// A tcgen05 MMA costs about the same for every N up to 128, so operands are stacked along N
+// wherever their products land in adjacent accumulator columns.
 // TMA brings q/k/v/g of the next chunk into the other half of a two-slot ring while a chunk is
 // processed.  Every wait is bounded; a time-out sets the workspace status to DS_TIMEOUT and the
 // CTA drains its copies, frees TMEM and returns.
@@ -39,40 +43,52 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kWaitLimit = 1u << 26;
 
-// TMEM columns (512 allocated)
-constexpr uint32_t TC_S = 0;       // state S, fp32 [Dv lanes][Dk cols]
-constexpr uint32_t TC_DELTA = 128; // U^T then Delta^T, fp32 [Dv][64 tokens]
-constexpr uint32_t TC_O = 192;     // O^T, fp32 [Dv][64 tokens]
-constexpr uint32_t TC_D = 256;     // intra D_0..D_3 (160 cols); later W^T (64 cols) and:
-constexpr uint32_t TC_SLO = 320;   //   bf16 lo part of the state operand (64 cols), phases 4b-5
-constexpr uint32_t TC_DLO = 384;   //   bf16 lo part of the Delta^T operand (32 cols), phases 6-7
-constexpr uint32_t TC_S0 = 416;    // bf16 state operand, 64 cols = 128 bf16 per lane
-constexpr uint32_t TC_DB = 480;    // bf16 Delta^T operand, 32 cols = 64 bf16 per lane
+// TMEM columns (512 allocated).  Lane = output row of every accumulator (dv for the state path).
+constexpr uint32_t TC_S = 0;      // state S, fp32 [Dv lanes][Dk cols]
+constexpr uint32_t TC_D = 128;    // phases 2-3: intra D_0..D_3 (160 cols)
+constexpr uint32_t TC_W = 128;    // phase 4: W^T partial products, Xsol_hi part | Xsol_lo part
+constexpr uint32_t TC_O = 128;    // phases 5-8: O^T [Dv][64 tokens]
+constexpr uint32_t TC_DA = 192;   // phase 5: S_hi (-W_hi)^T + S_lo (-W_hi)^T
+constexpr uint32_t TC_DB = 256;   // phase 5: S_hi (-W_lo)^T
+constexpr uint32_t TC_U = 320;    // phases 4-6: U^T
+constexpr uint32_t TC_SHI = 384;  // bf16 state operand hi (64 cols = 128 bf16 per lane)
+constexpr uint32_t TC_SLO = 448;  // bf16 state operand lo
+constexpr uint32_t TC_DHI = 384;  // phases 6-7: bf16 Delta^T operand hi (32 cols), over TC_SHI
+constexpr uint32_t TC_DLO = 416;  //              and its lo part
 
-// shared memory map (offsets from a 1024-byte aligned base)
+// Shared memory (offsets from a 1024-byte aligned base).  A ring slot holds one chunk's raw
+// tiles as 64-row x 64-column atoms (8 KB, 128-byte swizzled):
+//   q0 | g0 | v0 | q1 | g1 | v1 | k0 | k1      (x0 = columns 0-63, x1 = columns 64-127)
+// so that after phase 4 the 192 rows [Q~ ; -W_hi ; -W_lo] of each column half are contiguous:
+// one K-major N=192 operand for phase 5.
 constexpr uint32_t SLOT_BYTES = 65536;
-constexpr uint32_t OFF_Q = 0, OFF_K = 16384, OFF_G = 32768, OFF_V = 49152;
+constexpr uint32_t OFF_Q = 0, OFF_G = 8192, OFF_V = 16384, OFF_K = 49152;
+constexpr uint32_t QGV_ATOM = 24576;  // distance between the two column halves of q, g, v
+constexpr uint32_t K_ATOM = 8192;
 constexpr uint32_t SM_AOP = 131072;   // [128 rows][128] bf16, 2 atoms of 16 KB; after phase 2:
-constexpr uint32_t SM_KLO = SM_AOP;           //   K^ lo part [64][128] (16 KB)
-constexpr uint32_t SM_XWLO = SM_AOP + 16384;  //   Xsol lo part [64][64], then -W lo part [64][128]
-constexpr uint32_t SM_OSTG = SM_AOP;          //   phase 8: out tile [64 tokens][128] for the TMA store
-constexpr uint32_t SM_BT = 163840;    // [B^(0); B^(1); B^(2); B^(3)]: one 160-row tile; then the solve
-constexpr uint32_t BT_ROWS = 160;
-constexpr uint32_t SM_XSOL = 204800;  // [64][64] bf16
-constexpr uint32_t SM_AQK = 212992;   // [64][64] bf16
-constexpr uint32_t SM_WTOT = 221184;  // fp32 [8][128] warp totals of the gate cumsum
-constexpr uint32_t SM_REFG = 225280;  // fp32 [4][128]: G at rows 15, 31, 47, 63
-constexpr uint32_t SM_GC = 227328;    // fp32 [128]: 2^G_last
-constexpr uint32_t SM_BETA = 227840;  // fp32 [64]
-constexpr uint32_t SM_BAR = 228096;   // raw_full[2], mma
-constexpr uint32_t SM_TSLOT = 228128;
-constexpr uint32_t SM_FLAG = 228132;
-constexpr uint32_t SM_END = 228160;
+constexpr uint32_t SM_XSOL = SM_AOP;  //   [Xsol hi ; Xsol lo] 128 rows x 64 cols (16 KB)
+constexpr uint32_t SM_OSTG = SM_AOP;  //   phase 8: out tile [64 tokens][128] for the TMA store
+constexpr uint32_t SM_BT = 163840;    // [B^(0); B^(1); B^(2); B^(3)]: one 160-row tile; the solve
+constexpr uint32_t BT_ROWS = 160;     //   scratch in phase 3
+constexpr uint32_t SM_KLO = 204800;   // K^ lo part [64][128] (phases 2-7); phase 1: constants
+constexpr uint32_t SM_CST = SM_KLO;   //   fp32 [7][4 blocks][128]
+constexpr uint32_t SM_AQK = 221184;   // [64][64] bf16 (phases 3-7); phase 1: warp totals
+constexpr uint32_t SM_WTOT = SM_AQK;  //   fp32 [16 warps][128]
+constexpr uint32_t SM_GC = 229376;    // fp32 [128]: 2^G_last
+constexpr uint32_t SM_BETA = 229888;  // fp32 [64]
+constexpr uint32_t SM_BAR = 230144;   // raw_full[2], mma
+constexpr uint32_t SM_TSLOT = 230168;
+constexpr uint32_t SM_FLAG = 230172;
+constexpr uint32_t SM_PROD = 230176;  // the TMA producer's state (thread 0 only), 128 bytes
+constexpr uint32_t SM_END = 230304;
 constexpr size_t kFusedSmemBytes = SM_END + 1024;
+
+// per-(block, column) constants of the operand factorisation, indices into SM_CST
+enum : int { CST_REF = 0, CST_GE, CST_P2REF, CST_KFAC, CST_CDIAG, CST_C2, CST_C3, CST_N };
 
 // Phase timestamps for performance analysis (CTA 0, thread 0, first 64 chunks).
 #define KDA_TS(slot_)                                                        \
@@ -82,34 +98,54 @@ constexpr size_t kFusedSmemBytes = SM_END + 1024;
 
 __device__ __forceinline__ uint32_t dcol(int I) { return 8u * I * (I + 1); }
 
+// Byte offset of element (row, col) of a 64-row tile stored as two 64-column atoms `atom` bytes
+// apart (128-byte swizzle inside each atom).
+__device__ __forceinline__ uint32_t atom_off(uint32_t atom, uint32_t row, uint32_t col) {
+  return (col >> 6) * atom + row * 128u + ((((col & 63u) >> 3) ^ (row & 7u)) << 4) + (col & 7u) * 2u;
+}
+
 __device__ __forceinline__ bool plan_ok(const Params& p) {
   return p.plan[PH_MAGIC] == kPlanMagic && p.plan[PH_CHECKSUM] == p.plan_checksum &&
          p.plan[PH_UNITS] == p.n_units;
 }
 
-__device__ __forceinline__ void unpack8(const uint4 v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    f[2 * e] = __uint_as_float(w[e] << 16);
-    f[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-  }
+__device__ __forceinline__ void unpack4(const uint2 v, float (&f)[4]) {
+  f[0] = __uint_as_float(v.x << 16);
+  f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  f[2] = __uint_as_float(v.y << 16);
+  f[3] = __uint_as_float(v.y & 0xFFFF0000u);
 }
+__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
+  return make_uint2(pack_bf16(a, b), pack_bf16(c, d));
+}
+// the two floats of a packed bf16 pair (low half = first element)
+__device__ __forceinline__ float bf16_lo_of(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi_of(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
 }
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct Maps {
   CUtensorMap q, k, v, g, o;
 };
 
-// A unit's plan record as the producer keeps it in registers.
+// A unit's plan record as the producer keeps it.
 struct UnitRec {
   int b, h, hq, tok0, nch;
 };
+// The load schedule, kept in shared memory: the cursor (next (unit, chunk) of this CTA's stream,
+// chunks planned so far, the plan records of the current and next unit, read one unit ahead so
+// no global load sits on the issue path), written by thread 0 only; and the chunk whose tiles
+// go out during the current chunk, which ten warps read to issue one TMA box each.
+struct Producer {
+  int pu, pc;
+  uint32_t issued;
+  UnitRec cur, next;
+  int ld_valid, ld_c, ld_slot;
+  UnitRec ld_rec;
+};
+static_assert(sizeof(Producer) <= SM_END - SM_PROD, "producer state overflows its region");
 __device__ __forceinline__ UnitRec read_rec(const Params& p, int u) {
   UnitRec r{0, 0, 0, 0, 0};
   if (u < p.n_units) {
@@ -123,66 +159,34 @@ __device__ __forceinline__ UnitRec read_rec(const Params& p, int u) {
   return r;
 }
 
-// TMA of chunk c of unit `ur` into ring slot `slot` (all four tensors, two 64-column boxes each).
-__device__ void issue_chunk_loads(const Params& p, const Maps& m, uint32_t sbase, const UnitRec& ur,
-                                  int c, int slot) {
-  const int b = ur.b, h = ur.h, hq = ur.hq, tok0 = ur.tok0;
-  const uint32_t bar = sbase + SM_BAR + 8u * slot;
-  const uint32_t dst = sbase + slot * SLOT_BYTES;
-  mbar_arrive_expect_tx(bar, SLOT_BYTES);
+// Tensor coordinates of chunk c of unit `ur` for the q/k maps (qc) and the v/g/out maps (vc).
+__device__ __forceinline__ void chunk_coords(const Params& p, const UnitRec& ur, int c, int& qc1,
+                                             int& qc2, int& vc1, int& vc2) {
   const int t = c * kChunk;
-  int qc1, qc2, vc1, vc2;
   if (p.layout == KDA_LAYOUT_BNSD) {
-    qc1 = t; qc2 = b * p.Nqk + hq; vc1 = t; vc2 = b * p.Nv + h;
+    qc1 = t; qc2 = ur.b * p.Nqk + ur.hq; vc1 = t; vc2 = ur.b * p.Nv + ur.h;
   } else {
-    const int row = (p.layout == KDA_LAYOUT_BSND ? b * p.S : tok0) + t;
-    qc1 = hq; qc2 = row; vc1 = h; vc2 = row;
-  }
-#pragma unroll
-  for (int a = 0; a < 2; ++a) {
-    tma_load_3d(dst + OFF_Q + a * 8192, &m.q, bar, 64 * a, qc1, qc2);
-    tma_load_3d(dst + OFF_K + a * 8192, &m.k, bar, 64 * a, qc1, qc2);
-    tma_load_3d(dst + OFF_G + a * 8192, &m.g, bar, 64 * a, vc1, vc2);
-    tma_load_3d(dst + OFF_V + a * 8192, &m.v, bar, 64 * a, vc1, vc2);
+    const int row = (p.layout == KDA_LAYOUT_BSND ? ur.b * p.S : ur.tok0) + t;
+    qc1 = ur.hq; qc2 = row; vc1 = ur.h; vc2 = row;
   }
 }
 
-// Rows of D_BLK (row block BLK of the intra product) -> T (fp32, scaled by beta, strictly
-// lower, into Ts with pitch 68) for k rows, or Aqk (bf16, lower with diagonal, K-major) for
-// q rows.  The TMEM load is issued by the whole warp; only lanes in row block BLK write.
-template <int BLK>
-__device__ __forceinline__ void extract_block(uint32_t ta, int r, bool krow, float br, float* Ts,
-                                              uint8_t* aqk) {
-  constexpr int NC = BLK + 1;
-  constexpr int TP = 68;
-  uint32_t v[16 * NC];
-#pragma unroll
-  for (int ch = 0; ch < NC; ++ch)
-    tmem_ld16(ta + 8u * BLK * (BLK + 1) + 16 * ch, *reinterpret_cast<uint32_t(*)[16]>(v + 16 * ch));
-  tmem_wait_ld();
-  if ((r >> 4) != BLK) return;
-  if (krow) {
-#pragma unroll
-    for (int s0 = 0; s0 < 64; s0 += 4) {
-      float f[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int s = s0 + e;
-        f[e] = (s < 16 * NC && s < r) ? br * __uint_as_float(v[s < 16 * NC ? s : 0]) : 0.f;
-      }
-      *reinterpret_cast<float4*>(Ts + r * TP + s0) = make_float4(f[0], f[1], f[2], f[3]);
-    }
-  } else {
-#pragma unroll
-    for (int s0 = 0; s0 < 64; s0 += 8) {
-      float f[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int s = s0 + e;
-        f[e] = (s < 16 * NC && s <= r) ? __uint_as_float(v[s < 16 * NC ? s : 0]) : 0.f;
-      }
-      *reinterpret_cast<uint4*>(aqk + sw128_offset(64, r, s0)) = pack8(f);
-    }
+// TMA of one 64x64 box of chunk c into ring slot `slot`: box 0-1 q (column halves), 2-3 g,
+// 4-5 v, 6-7 k.  Every box arrives on the slot's barrier with its own byte count, so the eight
+// boxes can be issued by eight threads (a TMA issue occupies its thread for tens of cycles).
+__device__ __forceinline__ void issue_box(const Params& p, const Maps& m, uint32_t sbase,
+                                          const UnitRec& ur, int c, int slot, int box) {
+  int qc1, qc2, vc1, vc2;
+  chunk_coords(p, ur, c, qc1, qc2, vc1, vc2);
+  const uint32_t bar = sbase + SM_BAR + 8u * slot;
+  const uint32_t dst = sbase + slot * SLOT_BYTES;
+  const int half = box & 1;
+  mbar_arrive_expect_tx(bar, 8192);
+  switch (box >> 1) {
+    case 0: tma_load_3d(dst + OFF_Q + half * QGV_ATOM, &m.q, bar, 64 * half, qc1, qc2); break;
+    case 1: tma_load_3d(dst + OFF_G + half * QGV_ATOM, &m.g, bar, 64 * half, vc1, vc2); break;
+    case 2: tma_load_3d(dst + OFF_V + half * QGV_ATOM, &m.v, bar, 64 * half, vc1, vc2); break;
+    default: tma_load_3d(dst + OFF_K + half * K_ATOM, &m.k, bar, 64 * half, qc1, qc2); break;
   }
 }
 
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t wq = (uint32_t)(warp & 3) * 32u;  // TMEM lane quarter of this warp
   const uint32_t wlane = wq << 16;
-  const int wg = warp >> 2;
+  const int wg = warp >> 2;  // warpgroup 0..3: each covers all 128 TMEM lanes
 
   if (!plan_ok(p)) {
     if (tid == 0) atomicExch(p.status, DS_PLAN);
@@ -206,13 +210,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_mma = sbase + SM_BAR + 16;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_FLAG);
   float* wtot = reinterpret_cast<float*>(sm + SM_WTOT);
-  float* refg = reinterpret_cast<float*>(sm + SM_REFG);
+  float* cst = reinterpret_cast<float*>(sm + SM_CST);
   float* gcs = reinterpret_cast<float*>(sm + SM_GC);
   float* beta_s = reinterpret_cast<float*>(sm + SM_BETA);
 
   if (tid == 0) {
-    mbar_init(sbase + SM_BAR, 1);
-    mbar_init(sbase + SM_BAR + 8, 1);
+    mbar_init(sbase + SM_BAR, 8);  // one arrival per TMA box of the slot
+    mbar_init(sbase + SM_BAR + 8, 8);
     mbar_init(bar_mma, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -226,33 +230,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(sm + SM_TSLOT);
+  const uint32_t tl = tbase + wlane;  // this warp's TMEM lane quarter
 
   const int G_stride = gridDim.x;
-  // producer cursor (thread 0): next (unit, chunk) of this CTA's stream to load
-  // (plan records are read one unit ahead so no global load sits on the issue path)
-  int pu = blockIdx.x, pc = 0;
-  uint32_t issued = 0;
-  UnitRec prec{0, 0, 0, 0, 0}, nrec{0, 0, 0, 0, 0};
-  auto produce = [&]() {
-    if (pu >= p.n_units) return;
-    issue_chunk_loads(p, maps, sbase, prec, pc, issued & 1);
-    ++issued;
-    if (++pc == prec.nch) {
-      pc = 0;
-      pu += G_stride;
-      prec = nrec;
-      nrec = read_rec(p, pu + G_stride);
+  // Thread 0 issues every MMA and plans the loads; the TMA boxes are issued by other warps so no
+  // thread carries more than one or two.  Per chunk c (ring slot s): during the phase-2 MMAs
+  // thread 0 picks chunk c+2 (slot s again); lane 0 of warps 1-6 issue its q/g/v boxes in phase 7
+  // (q/g/v of slot s are free once the phase-5 MMAs are done), lane 0 of warps 7-8 its k boxes in
+  // phase 8 (after the phase-7 MMAs); lane 0 of warps 9-10 store chunk c's out tile after phase 8.
+  Producer* prod = reinterpret_cast<Producer*>(sm + SM_PROD);
+  auto plan_load = [&]() {  // thread 0
+    Producer& pr = *prod;
+    if (pr.pu >= p.n_units) {
+      pr.ld_valid = 0;
+      return;
+    }
+    pr.ld_valid = 1;
+    pr.ld_rec = pr.cur;
+    pr.ld_c = pr.pc;
+    pr.ld_slot = pr.issued & 1;
+    ++pr.issued;
+    if (++pr.pc == pr.cur.nch) {
+      pr.pc = 0;
+      pr.pu += G_stride;
+      pr.cur = pr.next;
+      pr.next = read_rec(p, pr.pu + G_stride);
     }
   };
+  auto issue_planned = [&](int box) {
+    const Producer& pr = *prod;
+    if (pr.ld_valid) issue_box(p, maps, sbase, pr.ld_rec, pr.ld_c, pr.ld_slot, box);
+  };
+  const bool st_thread = lane == 0 && (warp == 9 || warp == 10);  // out-tile store issuers
   if (tid == 0) {
-    prec = read_rec(p, pu);
-    nrec = read_rec(p, pu + G_stride);
+    prod->pu = blockIdx.x;
+    prod->pc = 0;
+    prod->issued = 0;
+    prod->cur = read_rec(p, blockIdx.x);
+    prod->next = read_rec(p, blockIdx.x + G_stride);
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.k);
     tma_prefetch_desc(&maps.v);
     tma_prefetch_desc(&maps.g);
-    produce();
-    produce();
+    tma_prefetch_desc(&maps.o);
+    for (int i = 0; i < 2; ++i) {  // chunks 0 and 1 of the stream
+      plan_load();
+      for (int box = 0; box < 8; ++box) issue_planned(box);
+    }
+    prod->ld_valid = 0;
   }
 
   uint32_t gidx = 0;       // chunks consumed by this CTA
@@ -268,6 +293,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_phase ^= 1u;
   };
 
+  // phase-1 thread map: warp w owns rows 4w..4w+3 (16-row block w/4), lane owns columns 4l..4l+3
+  const int r0 = 4 * warp, j0 = 4 * lane, Jb = warp >> 2;
+
   for (int u = blockIdx.x; u < p.n_units && !aborted; u += G_stride) {
     const int32_t* rec = p.plan + kPlanHeader + u * kPlanRecord;
     const int b = rec[PR_B], h = rec[PR_H], tok0 = rec[PR_TOK_START];
@@ -275,21 +303,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t sbase_g = ((size_t)b * p.Nv + h) * kD * kD;
     const float a_h = expf(p.A_log[h]);
     const float lbl2 = p.lower_bound * kLog2e;
-    const int cg = tid & 15, rg = tid >> 4;
-    const int j0 = cg * 8, r0 = rg * 4, Jb = rg >> 2;
-    float dtb[8];
+    float dtb[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dtb[e] = p.dt_bias[h * kD + j0 + e];
+    for (int e = 0; e < 4; ++e) dtb[e] = p.dt_bias[h * kD + j0 + e];
 
-    // ---- state from initial_state (fp32 -> TMEM S, bf16 -> TMEM S0) ----
+    // ---- state from initial_state: fp32 -> TMEM S, bf16 hi/lo -> TMEM state operand ----
     {
       const int i = wq + lane;
-#pragma unroll
+#pragma unroll 1
       for (int half = 0; half < 2; ++half) {
-        uint32_t fv[32];
-        const int col0 = wg * 64 + half * 32;
+        const int col0 = wg * 32 + half * 16;
+        uint32_t fv[16], hi[8], lo[8];
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
+        for (int c = 0; c < 16; c += 4) {
           float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
           if (p.S0) x = __ldg(reinterpret_cast<const float4*>(p.S0 + sbase_g + (size_t)i * kD + col0 + c));
           fv[c] = __float_as_uint(x.x);
@@ -297,38 +323,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           fv[c + 2] = __float_as_uint(x.z);
           fv[c + 3] = __float_as_uint(x.w);
         }
-        uint32_t lo[16], hi[16], pk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          lo[c] = fv[c];
-          hi[c] = fv[16 + c];
+        for (int c = 0; c < 8; ++c) {
+          const float x0 = __uint_as_float(fv[2 * c]), x1 = __uint_as_float(fv[2 * c + 1]);
+          hi[c] = pack_bf16(x0, x1);
+          lo[c] = pack_bf16(x0 - bf16_round(x0), x1 - bf16_round(x1));
         }
-        tmem_st16(tbase + wlane + TC_S + col0, lo);
-        tmem_st16(tbase + wlane + TC_S + col0 + 16, hi);
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = pack_bf16(__uint_as_float(fv[2 * c]), __uint_as_float(fv[2 * c + 1]));
-        tmem_st16(tbase + wlane + TC_S0 + col0 / 2, pk);
+        tmem_st16(tl + TC_S + col0, fv);
+        tmem_st8(tl + TC_SHI + col0 / 2, hi);
+        tmem_st8(tl + TC_SLO + col0 / 2, lo);
       }
       tmem_wait_st();
     }
     tc_fence_before();
     __syncthreads();
 
-    float bl_next = 0.f;
-    if (tid < kChunk && tid < L)
-      bl_next = __bfloat162float(p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, tid)]);
+    // beta logits of the next chunk (row tid), loaded one chunk ahead under the phase-5 MMAs
+    __nv_bfloat16 bl_next = __float2bfloat16_rn(0.f);
+    if (tid < kChunk && tid < L) bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, tid)];
 
     for (int c = 0; c < nch; ++c, ++gidx) {
       const int slot = gidx & 1;
-      uint8_t* sQ = sm + slot * SLOT_BYTES + OFF_Q;
-      uint8_t* sK = sm + slot * SLOT_BYTES + OFF_K;
-      uint8_t* sG = sm + slot * SLOT_BYTES + OFF_G;
-      uint8_t* sV = sm + slot * SLOT_BYTES + OFF_V;
-      const uint32_t aQ = sbase + slot * SLOT_BYTES + OFF_Q;
-      const uint32_t aK = sbase + slot * SLOT_BYTES + OFF_K;
-      const uint32_t aG = sbase + slot * SLOT_BYTES + OFF_G;
-      const uint32_t aV = sbase + slot * SLOT_BYTES + OFF_V;
+      uint8_t* sq = sm + slot * SLOT_BYTES;  // slot base: q, g, v atoms at QGV_ATOM, k at K_ATOM
+      const uint32_t as = sbase + slot * SLOT_BYTES;
       const int t0 = c * kChunk;
       const int n = min(kChunk, L - t0);
       const bool last = (c == nch - 1);
@@ -336,26 +353,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       KDA_TS(0);
 
       // =================== phase 1: prologue and operand tiles ===================
-      const float blog = bl_next;  // this chunk's beta logit (row tid), loaded one chunk ahead
-      if (c + 1 < nch && tid < kChunk && t0 + kChunk + tid < L)
-        bl_next = __bfloat162float(
-            p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t0 + kChunk + tid)]);
+      const __nv_bfloat16 blog = bl_next;
       if (!mbar_wait_bounded(sbase + SM_BAR + 8u * slot, (gidx >> 1) & 1u, kWaitLimit)) fail();
-      if (tid == 0) tma_store_wait_read();  // the out tile staged in the Aop region was read
       KDA_TS(1);
 
-      float G[4][8];
-      uint4 khlo[4];  // K^ lo parts of this thread's rows, stored once the intra MMA is done
+      float G[4][4];
       {
         // g_act * log2(e) = lb log2(e) / (1 + 2^(-log2(e) e^A_log (g_raw + dt_bias)))
         const float ca = -a_h * kLog2e;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = r0 + i;
-          float gv[8];
-          unpack8(*reinterpret_cast<const uint4*>(sG + sw128_offset(64, r, j0)), gv);
+          float gv[4];
+          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_G + atom_off(QGV_ATOM, r, j0)), gv);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 4; ++e) {
             const float sg = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
             G[i][e] = (r < n) ? sg : 0.0f;
           }
@@ -363,75 +375,71 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 1; i < 4; ++i)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) G[i][e] += G[i - 1][e];
+          for (int e = 0; e < 4; ++e) G[i][e] += G[i - 1][e];
+        *reinterpret_cast<float4*>(wtot + warp * kD + j0) =
+            make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
       }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float t = __shfl_up_sync(0xffffffffu, G[3][e], 16);
-        if (lane >= 16) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) G[i][e] += t;
-        }
-      }
-      if (lane >= 16) {
-        float4* dst = reinterpret_cast<float4*>(wtot + warp * kD + j0);
-        dst[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
-        dst[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
-      }
-      if (tid < kChunk) beta_s[tid] = (tid < n) ? __fdividef(1.0f, 1.0f + __expf(-blog)) : 0.0f;
+      if (tid < kChunk)
+        beta_s[tid] = (tid < n) ? __fdividef(1.0f, 1.0f + __expf(-__bfloat162float(blog))) : 0.0f;
       __syncthreads();
       KDA_TS(11);
-      {
-        float pre[8];
+      if (tid < kD) {
+        // column tid: exclusive prefix of the 16 warp totals (in place); the block reference rows
+        // (G at rows 15, 31, 47, 63) and from them the per-block constants of the factorisation
+        const int j = tid;
+        float run = 0.f, ref[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) pre[e] = 0.f;
-        for (int w2 = 0; w2 < warp; ++w2) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pre[e] += wtot[w2 * kD + j0 + e];
+        for (int w2 = 0; w2 < 16; ++w2) {
+          const float t = wtot[w2 * kD + j];
+          wtot[w2 * kD + j] = run;
+          run += t;
+          if ((w2 & 3) == 3) ref[w2 >> 2] = run;
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) G[i][e] += pre[e];
+        for (int I = 0; I < 4; ++I) {
+          const float refI = (I == 0) ? 0.f : ref[I - 1];
+          const float ge = ref[I];
+          cst[(CST_REF * 4 + I) * kD + j] = refI;
+          cst[(CST_GE * 4 + I) * kD + j] = ge;
+          cst[(CST_P2REF * 4 + I) * kD + j] = ex2(refI);
+          cst[(CST_KFAC * 4 + I) * kD + j] = ex2(ref[3] - ge);
+          cst[(CST_CDIAG * 4 + I) * kD + j] = ex2(refI - ge);
+          cst[(CST_C2 * 4 + I) * kD + j] = (I <= 1) ? ex2(ref[I + 1] - ge) : 0.f;
+          cst[(CST_C3 * 4 + I) * kD + j] = (I == 0) ? ex2(ref[2] - ge) : 0.f;
+        }
+        gcs[j] = ex2(ref[3]);
       }
-      if ((rg & 3) == 3) {
-        float4* dst = reinterpret_cast<float4*>(refg + Jb * kD + j0);
-        dst[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
-        dst[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
-      }
+      if (st_thread) tma_store_wait_read();  // the out tile staged in the Aop region was read
       __syncthreads();
       KDA_TS(12);
-      if (tid < kD) gcs[tid] = ex2(refg[3 * kD + tid]);
+      uint2 khlo[4];  // K^ lo parts of this thread's rows, stored once the intra MMA is done
       {
-        // reference rows of this thread's 16-row block Jb (read straight from shared memory so
-        // no register array is indexed by the thread-dependent block number)
-        const float* Rprev = refg + (Jb == 0 ? 0 : Jb - 1) * kD + j0;  // G at row 16 Jb - 1
-        const float* Rown = refg + Jb * kD + j0;                       // G at row 16 Jb + 15
-        const float* Rnext = refg + (Jb < 3 ? Jb + 1 : 3) * kD + j0;   // G at row 16 Jb + 31
-        const float* Rlast = refg + 3 * kD + j0;                       // G at row 63 (= G_last)
-        float refI[8], GeJ[8], p2ref[8], kfac[8], cdiag[8], c2[8], c3[8];
+        float k4[CST_N][4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          refI[e] = (Jb == 0) ? 0.f : Rprev[e];
-          GeJ[e] = Rown[e];
-          p2ref[e] = ex2(refI[e]);
-          kfac[e] = ex2(Rlast[e] - GeJ[e]);
-          cdiag[e] = ex2(refI[e] - GeJ[e]);
-          c2[e] = (Jb <= 1) ? ex2(Rnext[e] - GeJ[e]) : 0.f;
-          c3[e] = (Jb == 0) ? ex2(refg[2 * kD + j0 + e] - GeJ[e]) : 0.f;
+        for (int v = 0; v < CST_N; ++v) {
+          const float4 x = *reinterpret_cast<const float4*>(cst + (v * 4 + Jb) * kD + j0);
+          k4[v][0] = x.x;
+          k4[v][1] = x.y;
+          k4[v][2] = x.z;
+          k4[v][3] = x.w;
         }
-        uint4 qraw[4], kraw[4];
+        {
+          const float4 x = *reinterpret_cast<const float4*>(wtot + warp * kD + j0);
+          const float pre[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) G[i][e] += pre[e];
+        }
         float rqv[4], rkv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          qraw[i] = *reinterpret_cast<const uint4*>(sQ + sw128_offset(64, r0 + i, j0));
-          kraw[i] = *reinterpret_cast<const uint4*>(sK + sw128_offset(64, r0 + i, j0));
-          float qv[8], kv[8];
-          unpack8(qraw[i], qv);
-          unpack8(kraw[i], kv);
+          float qv[4], kv[4];
+          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r0 + i, j0)), qv);
+          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r0 + i, j0)), kv);
           float ssq = 0.f, ssk = 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 4; ++e) {
             ssq = fmaf(qv[e], qv[e], ssq);
             ssk = fmaf(kv[e], kv[e], ssk);
           }
@@ -439,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           rkv[i] = ssk;
         }
 #pragma unroll
-        for (int o = 1; o < 16; o <<= 1)
+        for (int o = 1; o < 32; o <<= 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             rqv[i] += __shfl_xor_sync(0xffffffffu, rqv[i], o);
@@ -449,45 +457,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const int r = r0 + i;
           const bool valid = r < n;
-          float qv[8], kv[8];
-          unpack8(qraw[i], qv);
-          unpack8(kraw[i], kv);
+          float qv[4], kv[4];
+          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j0)), qv);
+          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0)), kv);
           const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
           const float rk = rsqrtf(rkv[i] + 1e-6f);
-          float ka[8], qa[8], kt[8], qt[8], kh[8], khl[8], b0[8], b1[8], b2[8], b3[8];
+          float ka[4], qa[4], kt[4], qt[4], kh[4], khl[4], b0[4], b1[4], b2[4], b3[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 4; ++e) {
             const float Gv = G[i][e];
             const float kn = valid ? kv[e] * rk : 0.f;
             const float qn = valid ? qv[e] * rq : 0.f;
-            const float fA = ex2(Gv - refI[e]);
-            const float kbe = kn * ex2(GeJ[e] - Gv);
+            const float fA = ex2(Gv - k4[CST_REF][e]);
+            const float kbe = kn * ex2(k4[CST_GE][e] - Gv);
             ka[e] = kn * fA;
             qa[e] = qn * fA;
-            kt[e] = ka[e] * p2ref[e];
-            qt[e] = qa[e] * p2ref[e];
-            kh[e] = kbe * kfac[e];
+            kt[e] = ka[e] * k4[CST_P2REF][e];
+            qt[e] = qa[e] * k4[CST_P2REF][e];
+            kh[e] = kbe * k4[CST_KFAC][e];
             khl[e] = kh[e] - bf16_round(kh[e]);
-            b0[e] = kbe * cdiag[e];  // B^(Jb): diagonal block
-            b1[e] = kbe;             // B^(Jb+1): reference row is this block's last row
-            b2[e] = kbe * c2[e];     // B^(Jb+2)
-            b3[e] = kbe * c3[e];     // B^(Jb+3)
+            b0[e] = kbe * k4[CST_CDIAG][e];  // B^(Jb): diagonal block
+            b1[e] = kbe;                     // B^(Jb+1): reference row is this block's last row
+            b2[e] = kbe * k4[CST_C2][e];     // B^(Jb+2)
+            b3[e] = kbe * k4[CST_C3][e];     // B^(Jb+3)
           }
-          *reinterpret_cast<uint4*>(sm + SM_AOP + sw128_offset(128, r, j0)) = pack8(ka);
-          *reinterpret_cast<uint4*>(sm + SM_AOP + sw128_offset(128, 64 + r, j0)) = pack8(qa);
-          *reinterpret_cast<uint4*>(sQ + sw128_offset(64, r, j0)) = pack8(qt);
-          *reinterpret_cast<uint4*>(sK + sw128_offset(64, r, j0)) = pack8(kh);
-          khlo[i] = pack8(khl);
-          *reinterpret_cast<uint4*>(sG + sw128_offset(64, r, j0)) = pack8(kt);
-          *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb) + r, j0)) =
-              pack8(b0);
+          *reinterpret_cast<uint2*>(sm + SM_AOP + sw128_offset(128, r, j0)) = pack4(ka[0], ka[1], ka[2], ka[3]);
+          *reinterpret_cast<uint2*>(sm + SM_AOP + sw128_offset(128, 64 + r, j0)) = pack4(qa[0], qa[1], qa[2], qa[3]);
+          *reinterpret_cast<uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j0)) = pack4(qt[0], qt[1], qt[2], qt[3]);
+          *reinterpret_cast<uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0)) = pack4(kh[0], kh[1], kh[2], kh[3]);
+          khlo[i] = pack4(khl[0], khl[1], khl[2], khl[3]);
+          *reinterpret_cast<uint2*>(sq + OFF_G + atom_off(QGV_ATOM, r, j0)) = pack4(kt[0], kt[1], kt[2], kt[3]);
+          *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb) + r, j0)) =
+              pack4(b0[0], b0[1], b0[2], b0[3]);
           if (Jb + 1 <= 3)
-            *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 1) + r, j0)) = pack8(b1);
+            *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 1) + r, j0)) =
+                pack4(b1[0], b1[1], b1[2], b1[3]);
           if (Jb + 2 <= 3)
-            *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 2) + r, j0)) = pack8(b2);
+            *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 2) + r, j0)) =
+                pack4(b2[0], b2[1], b2[2], b2[3]);
           if (Jb + 3 <= 3)
-            *reinterpret_cast<uint4*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 3) + r, j0)) = pack8(b3);
-          if (!valid) *reinterpret_cast<uint4*>(sV + sw128_offset(64, r, j0)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 3) + r, j0)) =
+                pack4(b3[0], b3[1], b3[2], b3[3]);
+          if (!valid) *reinterpret_cast<uint2*>(sq + OFF_V + atom_off(QGV_ATOM, r, j0)) = make_uint2(0, 0);
         }
       }
       fence_proxy_async_smem();
@@ -502,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // =================== phase 2: intra MMAs ===================
       if (tid == 0) {
         tc_fence_after();
-        // D[:, 0:160] = Aop [B^(0); B^(1); B^(2); B^(3)]^T in one N=160 MMA chain: D_I = cols dcol(I)..
+        // D[:, 0:160] = Aop [B^(0); B^(1); B^(2); B^(3)]^T in one N=160 chain: D_I = cols dcol(I)..
         const uint32_t idesc = idesc_bf16(128, BT_ROWS, 0, 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -512,13 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tbase + TC_D, ad, bd, idesc, kk > 0);
         }
         mma_commit(bar_mma);
+        plan_load();  // the chunk after next, whose boxes go out in phases 7 and 8
       }
       wait_mma();
       KDA_TS(3);
       tc_fence_after();
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<uint4*>(sm + SM_KLO + sw128_offset(64, r0 + i, j0)) = khlo[i];
+        *reinterpret_cast<uint2*>(sm + SM_KLO + sw128_offset(64, r0 + i, j0)) = khlo[i];
 
       // =================== phase 3: T, Aqk, solve ===================
       // fp32 scratch in the B-tile region (free once the intra MMA has completed)
@@ -527,219 +539,366 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* Xs = Ts + 64 * TP;                           // X = (I + T)^-1            [64][TP]
       float* Ys = Xs + 64 * TP;                           // block products            [32][YP]
       {
-        // warp w: lane quarter q = w & 3 (q < 2: k rows -> T; q >= 2: q rows -> Aqk), row block
-        // blk = 2 (q & 1) + (w >> 2); one batched TMEM load of D_blk, then the 16 lanes of that
-        // block write their rows.  X is cleared alongside.
+        // TMEM lane quarter q4 = warp & 3 holds rows 32 (q4 & 1) .. +31 of k (q4 < 2) or q (q4 >= 2),
+        // i.e. row blocks bA = 2 (q4 & 1) and bA + 1.  The quarter's 8 items (block, 16-column
+        // chunk) are split over its 4 warps; chunks right of a block's diagonal are zero.
         const int q4 = warp & 3;
         const int r = (q4 & 1) * 32 + lane;
-        const int blk = 2 * (q4 & 1) + (warp >> 2);
         const bool krow = q4 < 2;
         const float br = krow ? beta_s[r] : 0.f;
-        const uint32_t ta = tbase + wlane + TC_D;
-        switch (blk) {
-          case 0: extract_block<0>(ta, r, krow, br, Ts, sm + SM_AQK); break;
-          case 1: extract_block<1>(ta, r, krow, br, Ts, sm + SM_AQK); break;
-          case 2: extract_block<2>(ta, r, krow, br, Ts, sm + SM_AQK); break;
-          default: extract_block<3>(ta, r, krow, br, Ts, sm + SM_AQK); break;
+        const int bA = 2 * (q4 & 1);
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int item = 2 * wg + it;
+          const int blk = bA + (item >> 2), ch = item & 3;
+          const bool mine = (r >> 4) == blk;
+          if (ch <= blk) {
+            uint32_t v[16];
+            tmem_ld16(tl + TC_D + dcol(blk) + 16 * ch, v);
+            tmem_wait_ld();
+            if (mine) {
+              if (krow) {
+#pragma unroll
+                for (int s0 = 0; s0 < 16; s0 += 4) {
+                  float f[4];
+#pragma unroll
+                  for (int e = 0; e < 4; ++e)
+                    f[e] = (16 * ch + s0 + e < r) ? br * __uint_as_float(v[s0 + e]) : 0.f;
+                  *reinterpret_cast<float4*>(Ts + r * TP + 16 * ch + s0) = make_float4(f[0], f[1], f[2], f[3]);
+                }
+              } else {
+#pragma unroll
+                for (int s0 = 0; s0 < 16; s0 += 8) {
+                  float f[8];
+#pragma unroll
+                  for (int e = 0; e < 8; ++e)
+                    f[e] = (16 * ch + s0 + e <= r) ? __uint_as_float(v[s0 + e]) : 0.f;
+                  *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch + s0)) = pack8(f);
+                }
+              }
+            }
+          } else if (mine && !krow) {
+            *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch + 8)) = make_uint4(0, 0, 0, 0);
+          }
         }
-        for (int e = tid; e < 64 * TP / 4; e += kThreads)
-          reinterpret_cast<float4*>(Xs)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        // the merges read strictly upper blocks of X that no level writes: X(0:16, 16:32) and
+        // X(32:48, 48:64) (16x16), and the upper 8x8 block of each 16x16 diagonal block
+        if (tid < 128) {
+          const int blk2 = tid >> 6, rr = (tid & 63) >> 2, c4 = (tid & 3) * 4;
+          *reinterpret_cast<float4*>(Xs + (32 * blk2 + rr) * TP + 32 * blk2 + 16 + c4) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        } else if (tid < 192) {
+          const int I = (tid - 128) >> 4, rr = ((tid - 128) >> 1) & 7, c4 = (tid & 1) * 4;
+          *reinterpret_cast<float4*>(Xs + (16 * I + rr) * TP + 16 * I + 8 + c4) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
       __syncthreads();
       KDA_TS(13);
-      // level 1: X_II = (I + T_II)^-1 for the four 16x16 diagonal blocks, one column per thread
+      // level 1a: X_mm = (I + T_mm)^-1 for the eight 8x8 diagonal blocks; thread = (block, column),
+      // rows by forward substitution as dot products over the already final entries
       if (tid < 64) {
-        const int I = tid >> 4, cc = tid & 15, base = 16 * I;
-        float x[16];
+        const int base = 8 * (tid >> 3), cc = tid & 7;
+        float x[8];
+        x[0] = (cc == 0) ? 1.f : 0.f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) x[k] = (k == cc) ? 1.f : 0.f;
-        // outer-product order: once x[k] is final, update every later row (independent FMAs)
+        for (int rr = 1; rr < 8; ++rr) {
+          const float* trow = Ts + (base + rr) * TP + base;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 15; ++k) {
+          for (int k0 = 0; k0 < rr; k0 += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
+            const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
-          for (int rr = k + 1; rr < 16; ++rr) x[rr] = fmaf(-Ts[(base + rr) * TP + base + k], x[k], x[rr]);
+            for (int e = 0; e < 4; ++e)
+              if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
+          }
+          const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
         }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) Xs[(base + k) * TP + base + cc] = x[k];
+        for (int k = 0; k < 8; ++k) Xs[(base + k) * TP + base + cc] = x[k];
+      }
+      __syncthreads();
+      // level 1b: X_(16I+8.., 16I..) = -X22 T21 X11 inside each 16x16 diagonal block (8x8 merges)
+      {
+        const int I = (tid >> 6) & 3, rr = (tid >> 3) & 7, cc = tid & 7;
+        const bool act = tid < 256;
+        const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
+        if (act) {
+          const float4 ta = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1);
+          const float4 tb = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1 + 4);
+          const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+          float y = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) y = fmaf(tv[k], Xs[(c1 + k) * TP + c1 + cc], y);
+          Ys[(8 * I + rr) * YP + cc] = y;
+        }
+        __syncthreads();
+        if (act) {
+          const float4 xa = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 8);
+          const float4 xb = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 12);
+          const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+          float z = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) z = fmaf(xv[k], Ys[(8 * I + k) * YP + cc], z);
+          Xs[r1 * TP + c1 + cc] = -z;
+        }
       }
       __syncthreads();
       KDA_TS(14);
-      // level 2: X_{I,I-1} = -X_II T_{I,I-1} X_{I-1,I-1} for I = 1, 3 (two 16x16 merges)
+      // level 2: X_{I,I-1} = -X_II T_{I,I-1} X_{I-1,I-1} for I = 1, 3 (two 16x16 merges).  A thread
+      // owns a 2x2 output tile and a quarter of the inner dimension; the quarters meet by shuffles.
       {
-        const int pI = tid >> 7, rr = (tid >> 3) & 15, c0 = (tid & 7) * 2;
+        const int kq = lane & 3, tile = warp * 8 + (lane >> 2);
+        const int pI = tile >> 6, tr = (tile >> 3) & 7, tc = tile & 7;
         const int I = 2 * pI + 1, J = I - 1;
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float t = Ts[(16 * I + rr) * TP + 16 * J + k];
-          const float2 xv = *reinterpret_cast<const float2*>(Xs + (16 * J + k) * TP + 16 * J + c0);
-          y0 = fmaf(t, xv.x, y0);
-          y1 = fmaf(t, xv.y, y1);
-        }
-        *reinterpret_cast<float2*>(Ys + (16 * pI + rr) * YP + c0) = make_float2(y0, y1);
-        __syncthreads();
-        float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float xx = Xs[(16 * I + rr) * TP + 16 * I + k];
-          const float2 yv = *reinterpret_cast<const float2*>(Ys + (16 * pI + k) * YP + c0);
-          z0 = fmaf(xx, yv.x, z0);
-          z1 = fmaf(xx, yv.y, z1);
-        }
-        *reinterpret_cast<float2*>(Xs + (16 * I + rr) * TP + 16 * J + c0) = make_float2(-z0, -z1);
-      }
-      __syncthreads();
-      KDA_TS(15);
-      // level 3: X_(32:64, 0:32) = -X_(32:64, 32:64) T_(32:64, 0:32) X_(0:32, 0:32) (32x32 merge);
-      // each thread owns a 2x2 output tile (rows 2 tr, 2 tr + 1; columns 2 tc, 2 tc + 1)
-      {
-        const int tr = tid >> 4, tc = tid & 15;
+        const int ra = 16 * I + 2 * tr, cb = 2 * tc;
         float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
-        for (int k0 = 0; k0 < 32; k0 += 4) {
-          const float4 ta = *reinterpret_cast<const float4*>(Ts + (32 + 2 * tr) * TP + k0);
-          const float4 tb = *reinterpret_cast<const float4*>(Ts + (33 + 2 * tr) * TP + k0);
+        {
+          const float4 ta = *reinterpret_cast<const float4*>(Ts + ra * TP + 16 * J + 4 * kq);
+          const float4 tb = *reinterpret_cast<const float4*>(Ts + (ra + 1) * TP + 16 * J + 4 * kq);
           const float tav[4] = {ta.x, ta.y, ta.z, ta.w}, tbv[4] = {tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 xv = *reinterpret_cast<const float2*>(Xs + (k0 + e) * TP + 2 * tc);
+            const float2 xv = *reinterpret_cast<const float2*>(Xs + (16 * J + 4 * kq + e) * TP + 16 * J + cb);
             y00 = fmaf(tav[e], xv.x, y00);
             y01 = fmaf(tav[e], xv.y, y01);
             y10 = fmaf(tbv[e], xv.x, y10);
             y11 = fmaf(tbv[e], xv.y, y11);
           }
         }
-        *reinterpret_cast<float2*>(Ys + (2 * tr) * YP + 2 * tc) = make_float2(y00, y01);
-        *reinterpret_cast<float2*>(Ys + (2 * tr + 1) * YP + 2 * tc) = make_float2(y10, y11);
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+          y00 += __shfl_xor_sync(0xffffffffu, y00, o);
+          y01 += __shfl_xor_sync(0xffffffffu, y01, o);
+          y10 += __shfl_xor_sync(0xffffffffu, y10, o);
+          y11 += __shfl_xor_sync(0xffffffffu, y11, o);
+        }
+        if (kq == 0) {
+          *reinterpret_cast<float2*>(Ys + (16 * pI + 2 * tr) * YP + cb) = make_float2(y00, y01);
+          *reinterpret_cast<float2*>(Ys + (16 * pI + 2 * tr + 1) * YP + cb) = make_float2(y10, y11);
+        }
         __syncthreads();
         float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
-#pragma unroll
-        for (int k0 = 0; k0 < 32; k0 += 4) {
-          const float4 xa = *reinterpret_cast<const float4*>(Xs + (32 + 2 * tr) * TP + 32 + k0);
-          const float4 xb = *reinterpret_cast<const float4*>(Xs + (33 + 2 * tr) * TP + 32 + k0);
+        {
+          const float4 xa = *reinterpret_cast<const float4*>(Xs + ra * TP + 16 * I + 4 * kq);
+          const float4 xb = *reinterpret_cast<const float4*>(Xs + (ra + 1) * TP + 16 * I + 4 * kq);
           const float xav[4] = {xa.x, xa.y, xa.z, xa.w}, xbv[4] = {xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 yv = *reinterpret_cast<const float2*>(Ys + (k0 + e) * YP + 2 * tc);
+            const float2 yv = *reinterpret_cast<const float2*>(Ys + (16 * pI + 4 * kq + e) * YP + cb);
             z00 = fmaf(xav[e], yv.x, z00);
             z01 = fmaf(xav[e], yv.y, z01);
             z10 = fmaf(xbv[e], yv.x, z10);
             z11 = fmaf(xbv[e], yv.y, z11);
           }
         }
-        *reinterpret_cast<float2*>(Xs + (32 + 2 * tr) * TP + 2 * tc) = make_float2(-z00, -z01);
-        *reinterpret_cast<float2*>(Xs + (33 + 2 * tr) * TP + 2 * tc) = make_float2(-z10, -z11);
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+          z00 += __shfl_xor_sync(0xffffffffu, z00, o);
+          z01 += __shfl_xor_sync(0xffffffffu, z01, o);
+          z10 += __shfl_xor_sync(0xffffffffu, z10, o);
+          z11 += __shfl_xor_sync(0xffffffffu, z11, o);
+        }
+        if (kq == 0) {
+          *reinterpret_cast<float2*>(Xs + ra * TP + 16 * J + cb) = make_float2(-z00, -z01);
+          *reinterpret_cast<float2*>(Xs + (ra + 1) * TP + 16 * J + cb) = make_float2(-z10, -z11);
+        }
+      }
+      __syncthreads();
+      KDA_TS(15);
+      // level 3: X_(32:64, 0:32) = -X_(32:64, 32:64) T_(32:64, 0:32) X_(0:32, 0:32) (32x32 merge).
+      // A thread owns a 4x2 output tile and the inner indices 4 kq + e + 16 m (e < 4, m < 2): the
+      // four kq of a warp read rows 4 apart, two 16-bank halves, so each load is 2 wavefronts.
+      {
+        const int kq = lane & 3, tile = warp * 8 + (lane >> 2);
+        const int ra = 32 + 4 * (tile >> 4), cb = 2 * (tile & 15);
+        float acc[4][2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const int kb = 4 * kq + 16 * m;
+          float tv[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 t4 = *reinterpret_cast<const float4*>(Ts + (ra + i) * TP + kb);
+            tv[i][0] = t4.x; tv[i][1] = t4.y; tv[i][2] = t4.z; tv[i][3] = t4.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 xv = *reinterpret_cast<const float2*>(Xs + (kb + e) * TP + cb);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[i][0] = fmaf(tv[i][e], xv.x, acc[i][0]);
+              acc[i][1] = fmaf(tv[i][e], xv.y, acc[i][1]);
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[i][0] += __shfl_xor_sync(0xffffffffu, acc[i][0], o);
+            acc[i][1] += __shfl_xor_sync(0xffffffffu, acc[i][1], o);
+          }
+        if (kq == 0) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float2*>(Ys + (ra - 32 + i) * YP + cb) = make_float2(acc[i][0], acc[i][1]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const int kb = 4 * kq + 16 * m;
+          float xv4[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 x4 = *reinterpret_cast<const float4*>(Xs + (ra + i) * TP + 32 + kb);
+            xv4[i][0] = x4.x; xv4[i][1] = x4.y; xv4[i][2] = x4.z; xv4[i][3] = x4.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 yv = *reinterpret_cast<const float2*>(Ys + (kb + e) * YP + cb);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[i][0] = fmaf(xv4[i][e], yv.x, acc[i][0]);
+              acc[i][1] = fmaf(xv4[i][e], yv.y, acc[i][1]);
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[i][0] += __shfl_xor_sync(0xffffffffu, acc[i][0], o);
+            acc[i][1] += __shfl_xor_sync(0xffffffffu, acc[i][1], o);
+          }
+        if (kq == 0) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float2*>(Xs + (ra + i) * TP + cb) = make_float2(-acc[i][0], -acc[i][1]);
+        }
       }
       __syncthreads();
       KDA_TS(16);
-      // Xsol = X diag(beta) -> bf16 hi and lo parts, K-major [r][s]
+      // Xsol = X diag(beta) -> bf16 hi (rows 0-63) and lo (rows 64-127) parts, K-major [r][s]
       {
-        const int r = tid >> 2, s0 = (tid & 3) * 16;
+        const int r = tid >> 3, s0 = (tid & 7) * 8;
+        const float4 xa = *reinterpret_cast<const float4*>(Xs + r * TP + s0);
+        const float4 xb = *reinterpret_cast<const float4*>(Xs + r * TP + s0 + 4);
+        const float4 ba = *reinterpret_cast<const float4*>(beta_s + s0);
+        const float4 bb = *reinterpret_cast<const float4*>(beta_s + s0 + 4);
+        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        const float bv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+        float f[8], fl[8];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float f[8], fl[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int s = s0 + 8 * hh + e;
-            f[e] = (s <= r) ? Xs[r * TP + s] * beta_s[s] : 0.f;
-            fl[e] = f[e] - bf16_round(f[e]);
-          }
-          *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(64, r, s0 + 8 * hh)) = pack8(f);
-          *reinterpret_cast<uint4*>(sm + SM_XWLO + sw128_offset(64, r, s0 + 8 * hh)) = pack8(fl);
+        for (int e = 0; e < 8; ++e) {
+          f[e] = (s0 + e <= r) ? xv[e] * bv[e] : 0.f;
+          fl[e] = f[e] - bf16_round(f[e]);
         }
+        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, r, s0)) = pack8(f);
+        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, 64 + r, s0)) = pack8(fl);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
       KDA_TS(4);
 
-      // =================== phase 4: W^T and U^T ===================
+      // =================== phase 4: W^T and U^T;  S <- S Diag(2^G_last) ===================
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, 64, 1, 0);
-        // W first (its epilogue waits on this commit), then U (consumed in order by phase 5)
+        // K~ and V are MN-major A operands (rows = tokens s, the two column halves QGV_ATOM apart)
+        const uint32_t idesc_w = idesc_bf16(128, 128, 1, 0);
+        const uint32_t idesc_u = idesc_bf16(128, 64, 1, 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t aw = smem_desc(aG + kk * 2048, 8192, 1024);
-          mma_ss(tbase + TC_D, aw, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc, kk > 0);
-          mma_ss(tbase + TC_D, aw, smem_desc(sbase + SM_XWLO + kk * 32, 16, 1024), idesc, 1);
+          const uint64_t aw = smem_desc(as + OFF_G + kk * 2048, QGV_ATOM, 1024);
+          mma_ss(tbase + TC_W, aw, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc_w, kk > 0);
         }
-        if (!dbg) mma_commit(bar_mma);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t av = smem_desc(aV + kk * 2048, 8192, 1024);
-          mma_ss(tbase + TC_DELTA, av, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc, kk > 0);
-          mma_ss(tbase + TC_DELTA, av, smem_desc(sbase + SM_XWLO + kk * 32, 16, 1024), idesc, 1);
+          const uint64_t av = smem_desc(as + OFF_V + kk * 2048, QGV_ATOM, 1024);
+          mma_ss(tbase + TC_U, av, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc_u, kk > 0);
+          mma_ss(tbase + TC_U, av, smem_desc(sbase + SM_XSOL + 8192 + kk * 32, 16, 1024), idesc_u, 1);
         }
-        if (dbg) mma_commit(bar_mma);  // the debug dump reads U too
+        mma_commit(bar_mma);
       }
       {
-        // lo part of the bf16 state operand, S - bf16(S), built while the W/U MMAs run (they
-        // touch neither TC_S nor TC_SLO)
+        // the state decay for this chunk (the phase-5 MMAs read the bf16 copies, not TC_S)
+        uint32_t v[16], w2[16];
+        const int col = wg * 32;
+        tmem_ld16(tl + TC_S + col, v);
+        tmem_ld16(tl + TC_S + col + 16, w2);
+        tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t v0[16], v1[16], pk[16];
-          const int col = wg * 64 + 32 * ch;
-          tmem_ld16(tbase + wlane + TC_S + col, v0);
-          tmem_ld16(tbase + wlane + TC_S + col + 16, v1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float a0 = __uint_as_float(v0[2 * e]), a1 = __uint_as_float(v0[2 * e + 1]);
-            const float c0 = __uint_as_float(v1[2 * e]), c1 = __uint_as_float(v1[2 * e + 1]);
-            pk[e] = pack_bf16(a0 - bf16_round(a0), a1 - bf16_round(a1));
-            pk[8 + e] = pack_bf16(c0 - bf16_round(c0), c1 - bf16_round(c1));
-          }
-          tmem_st16(tbase + wlane + TC_SLO + col / 2, pk);
+        for (int e4 = 0; e4 < 16; e4 += 4) {
+          const float4 ga = *reinterpret_cast<const float4*>(gcs + col + e4);
+          const float4 gb = *reinterpret_cast<const float4*>(gcs + col + 16 + e4);
+          v[e4] = __float_as_uint(__uint_as_float(v[e4]) * ga.x);
+          v[e4 + 1] = __float_as_uint(__uint_as_float(v[e4 + 1]) * ga.y);
+          v[e4 + 2] = __float_as_uint(__uint_as_float(v[e4 + 2]) * ga.z);
+          v[e4 + 3] = __float_as_uint(__uint_as_float(v[e4 + 3]) * ga.w);
+          w2[e4] = __float_as_uint(__uint_as_float(w2[e4]) * gb.x);
+          w2[e4 + 1] = __float_as_uint(__uint_as_float(w2[e4 + 1]) * gb.y);
+          w2[e4 + 2] = __float_as_uint(__uint_as_float(w2[e4 + 2]) * gb.z);
+          w2[e4 + 3] = __float_as_uint(__uint_as_float(w2[e4 + 3]) * gb.w);
         }
+        tmem_st16(tl + TC_S + col, v);
+        tmem_st16(tl + TC_S + col + 16, w2);
         tmem_wait_st();
       }
       wait_mma();
       KDA_TS(5);
       tc_fence_after();
       {
-        // W^T row j (tokens r = 32 wg .. 32 wg + 31) -> -W^T stored MN-major: tile [j][r], one atom
+        // W row r (r = 16 wg .. 16 wg + 15) at lane j: -W -> bf16 hi over the K~ tile, lo over the
+        // V tile, token-major [r][j] (the K-major layout of the phase-5 B operand).  Lanes j and
+        // j ^ 1 swap one value per row pair, so each writes two adjacent columns of one row.
         const int j = wq + lane;
-        uint32_t vw[2][16];
-        tmem_ld16(tbase + wlane + TC_D + wg * 32, vw[0]);
-        tmem_ld16(tbase + wlane + TC_D + wg * 32 + 16, vw[1]);
+        const bool odd = lane & 1;
+        uint32_t va[16], vb[16];
+        tmem_ld16(tl + TC_W + 16 * wg, va);
+        tmem_ld16(tl + TC_W + 64 + 16 * wg, vb);
         tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const uint32_t* v = vw[ch];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            float hi[8], lo[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float wv = -__uint_as_float(v[8 * hh + e]);
-              hi[e] = wv;
-              lo[e] = wv - bf16_round(wv);
-            }
-            const int rc = wg * 32 + 16 * ch + 8 * hh;  // first token of this 8-wide chunk
-            *reinterpret_cast<uint4*>(sG + sw128_offset(128, j, rc)) = pack8(hi);
-            *reinterpret_cast<uint4*>(sm + SM_XWLO + sw128_offset(128, j, rc)) = pack8(lo);
-          }
+        for (int q = 0; q < 8; ++q) {
+          const float w0 = -(__uint_as_float(va[2 * q]) + __uint_as_float(vb[2 * q]));
+          const float w1 = -(__uint_as_float(va[2 * q + 1]) + __uint_as_float(vb[2 * q + 1]));
+          const float recv = __shfl_xor_sync(0xffffffffu, odd ? w0 : w1, 1);
+          const float x0 = odd ? recv : w0, x1 = odd ? w1 : recv;  // columns j & ~1 and j | 1
+          const int r = 16 * wg + 2 * q + (odd ? 1 : 0);
+          const uint32_t off = atom_off(QGV_ATOM, r, j & ~1);
+          const uint32_t hi = pack_bf16(x0, x1);
+          const uint32_t lo = pack_bf16(x0 - bf16_lo_of(hi), x1 - bf16_hi_of(hi));
+          *reinterpret_cast<uint32_t*>(sq + OFF_G + off) = hi;
+          *reinterpret_cast<uint32_t*>(sq + OFF_V + off) = lo;
         }
       }
       if (dbg) {  // per-chunk intermediates in the two-kernel workspace layout (fp32)
         float* dc = dbg + (size_t)(coff + c) * (kWsChunkBytes / 4);
         const int i = wq + lane;
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t v[16], w[16];
-          tmem_ld16(tbase + wlane + TC_D + 16 * ch, w);
-          tmem_ld16(tbase + wlane + TC_DELTA + 16 * ch, v);
-          tmem_wait_ld();
-          if (wg == 0)
+        if (wg == 0) {
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t wa[16], wb[16], v[16];
+            tmem_ld16(tl + TC_W + 16 * ch, wa);
+            tmem_ld16(tl + TC_W + 64 + 16 * ch, wb);
+            tmem_ld16(tl + TC_U + 16 * ch, v);
+            tmem_wait_ld();
             for (int e = 0; e < 16; ++e) {
-              dc[kWsW / 4 + (16 * ch + e) * kD + i] = __uint_as_float(w[e]);
+              dc[kWsW / 4 + (16 * ch + e) * kD + i] = __uint_as_float(wa[e]) + __uint_as_float(wb[e]);
               dc[kWsU / 4 + (16 * ch + e) * kD + i] = __uint_as_float(v[e]);
             }
+          }
         }
         for (int e = tid; e < kChunk * kD; e += kThreads) {
           const int r = e / kD, j = e % kD;
-          dc[kWsQt / 4 + e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sQ + sw128_offset(64, r, j)));
-          dc[kWsKh / 4 + e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sK + sw128_offset(64, r, j)));
+          dc[kWsQt / 4 + e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j)));
+          dc[kWsKh / 4 + e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sq + OFF_K + atom_off(K_ATOM, r, j)));
         }
         for (int e = tid; e < kChunk * kChunk; e += kThreads) {
           const int r = e / kChunk, s = e % kChunk;
@@ -752,68 +911,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       KDA_TS(6);
 
-      // =================== phase 5: Delta^T = U^T - S0 W^T,  O^T = S0 Q~^T ===================
+      // ============ phase 5: [O^T | Da | Db] = S [Q~ | -W_hi | -W_lo]^T ============
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, 64, 0, 0);
-        const uint32_t idesc_w = idesc_bf16(128, 64, 0, 1);  // -W^T tiles are MN-major [j][r]
-        // Delta first (phase 6 waits on this commit); O^T = S0 Q~^T after it, covered by the
-        // commit of phase 7
+        // B rows: Q~ (0-63), -W_hi (64-127), -W_lo (128-191): one K-major tile per column half
+        const uint32_t idesc_3 = idesc_bf16(128, 192, 0, 0);
+        const uint32_t idesc_2 = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bw = smem_desc(aG + kk * 2048, 16384, 1024);
-          mma_ts(tbase + TC_DELTA, tbase + TC_S0 + kk * 8, bw, idesc_w, 1);
-          mma_ts(tbase + TC_DELTA, tbase + TC_SLO + kk * 8, bw, idesc_w, 1);
-          mma_ts(tbase + TC_DELTA, tbase + TC_S0 + kk * 8,
-                 smem_desc(sbase + SM_XWLO + kk * 2048, 16384, 1024), idesc_w, 1);
+          const uint64_t bd = smem_desc(as + (kk >> 2) * QGV_ATOM + (kk & 3) * 32, 16, 1024);
+          mma_ts(tbase + TC_O, tbase + TC_SHI + kk * 8, bd, idesc_3, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = smem_desc(as + (kk >> 2) * QGV_ATOM + (kk & 3) * 32, 16, 1024);
+          mma_ts(tbase + TC_O, tbase + TC_SLO + kk * 8, bd, idesc_2, 1);
         }
         mma_commit(bar_mma);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-          mma_ts(tbase + TC_O, tbase + TC_S0 + kk * 8, smem_desc(aQ + koff, 16, 1024), idesc, kk > 0);
-        }
       }
-      if (wg == 1) {
-        // S <- S Diag(2^G_last) while the Delta/O MMAs run (they read the bf16 copies, not TC_S)
-#pragma unroll
-        for (int ch = 0; ch < 8; ch += 2) {
-          uint32_t v[16], w2[16];
-          tmem_ld16(tbase + wlane + TC_S + 16 * ch, v);
-          tmem_ld16(tbase + wlane + TC_S + 16 * ch + 16, w2);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            v[e] = __float_as_uint(__uint_as_float(v[e]) * gcs[16 * ch + e]);
-            w2[e] = __float_as_uint(__uint_as_float(w2[e]) * gcs[16 * ch + 16 + e]);
-          }
-          tmem_st16(tbase + wlane + TC_S + 16 * ch, v);
-          tmem_st16(tbase + wlane + TC_S + 16 * ch + 16, w2);
-        }
-        tmem_wait_st();
-      }
+      if (c + 1 < nch && tid < kChunk && t0 + kChunk + tid < L)
+        bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t0 + kChunk + tid)];
       wait_mma();
       KDA_TS(7);
       tc_fence_after();
 
-      // =================== phase 6: Delta^T -> bf16 hi and lo ===================
+      // =================== phase 6: Delta^T = U^T + Da + Db -> bf16 hi and lo ===================
       {
-        // warpgroup wg converts tokens 32 wg .. 32 wg + 31 (one batched load of 32 columns)
-        uint32_t v0[16], v1[16], hi[16], lo[16];
-        tmem_ld16(tbase + wlane + TC_DELTA + 32 * wg, v0);
-        tmem_ld16(tbase + wlane + TC_DELTA + 32 * wg + 16, v1);
+        // warpgroup wg converts tokens 16 wg .. 16 wg + 15
+        uint32_t va[16], vb[16], vu[16], hi[8], lo[8];
+        tmem_ld16(tl + TC_DA + 16 * wg, va);
+        tmem_ld16(tl + TC_DB + 16 * wg, vb);
+        tmem_ld16(tl + TC_U + 16 * wg, vu);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float d0 = __uint_as_float(v0[2 * e]), d1 = __uint_as_float(v0[2 * e + 1]);
-          const float d2 = __uint_as_float(v1[2 * e]), d3 = __uint_as_float(v1[2 * e + 1]);
+          const float d0 = __uint_as_float(vu[2 * e]) + __uint_as_float(va[2 * e]) + __uint_as_float(vb[2 * e]);
+          const float d1 = __uint_as_float(vu[2 * e + 1]) + __uint_as_float(va[2 * e + 1]) +
+                           __uint_as_float(vb[2 * e + 1]);
           hi[e] = pack_bf16(d0, d1);
-          hi[8 + e] = pack_bf16(d2, d3);
           lo[e] = pack_bf16(d0 - bf16_round(d0), d1 - bf16_round(d1));
-          lo[8 + e] = pack_bf16(d2 - bf16_round(d2), d3 - bf16_round(d3));
         }
-        tmem_st16(tbase + wlane + TC_DB + 16 * wg, hi);
-        tmem_st16(tbase + wlane + TC_DLO + 16 * wg, lo);
+        tmem_st8(tl + TC_DHI + 8 * wg, hi);
+        tmem_st8(tl + TC_DLO + 8 * wg, lo);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -827,80 +966,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t idesc_o = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bk = smem_desc(aK + kk * 2048, 8192, 1024);
-          mma_ts(tbase + TC_S, tbase + TC_DB + kk * 8, bk, idesc_s, 1);
+          const uint64_t bk = smem_desc(as + OFF_K + kk * 2048, K_ATOM, 1024);
+          mma_ts(tbase + TC_S, tbase + TC_DHI + kk * 8, bk, idesc_s, 1);
           mma_ts(tbase + TC_S, tbase + TC_DLO + kk * 8, bk, idesc_s, 1);
-          mma_ts(tbase + TC_S, tbase + TC_DB + kk * 8, smem_desc(sbase + SM_KLO + kk * 2048, 8192, 1024),
+          mma_ts(tbase + TC_S, tbase + TC_DHI + kk * 8, smem_desc(sbase + SM_KLO + kk * 2048, 8192, 1024),
                  idesc_s, 1);
-          mma_ts(tbase + TC_O, tbase + TC_DB + kk * 8, smem_desc(sbase + SM_AQK + kk * 32, 16, 1024),
+          mma_ts(tbase + TC_O, tbase + TC_DHI + kk * 8, smem_desc(sbase + SM_AQK + kk * 32, 16, 1024),
                  idesc_o, 1);
         }
         mma_commit(bar_mma);
       }
+      if (lane == 0 && warp >= 1 && warp <= 6) issue_planned(warp - 1);  // q/g/v of this slot are free
       wait_mma();
       KDA_TS(9);
-      if (tid == 0 && !*abort_flag) {
-        fence_proxy_async_smem();
-        produce();  // the slot of this chunk is free: bring in the chunk after next
-      }
-      KDA_TS(17);
       tc_fence_after();
+      if (lane == 0 && (warp == 7 || warp == 8)) issue_planned(warp - 1);  // and now its k tile
 
       // =================== phase 8: out rows;  S -> bf16 operand (and final_state) ===================
       {
         const int i = wq + lane;
-        uint32_t vo[2][16];
-        tmem_ld16(tbase + wlane + TC_O + wg * 32, vo[0]);
-        tmem_ld16(tbase + wlane + TC_O + wg * 32 + 16, vo[1]);
+        uint32_t vo[16];
+        tmem_ld16(tl + TC_O + 16 * wg, vo);
         tmem_wait_ld();
         if (n == kChunk) {
           // full chunk: out tile [t][i] (128B-swizzled, as the out tensor map expects) in the free
-          // Aop region, then two TMA stores issued below
+          // Aop region, stored by TMA after the phase-8 barrier
+          // (lanes i and i ^ 1 swap one value per token pair and write two adjacent columns)
+          const bool odd = lane & 1;
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int t = wg * 32 + 16 * ch + e;
-              *reinterpret_cast<__nv_bfloat16*>(sm + SM_OSTG + sw128_offset(64, t, i)) =
-                  __float2bfloat16_rn(__uint_as_float(vo[ch][e]));
-            }
+          for (int q = 0; q < 8; ++q) {
+            const float o0 = __uint_as_float(vo[2 * q]), o1 = __uint_as_float(vo[2 * q + 1]);
+            const float recv = __shfl_xor_sync(0xffffffffu, odd ? o0 : o1, 1);
+            const int t = 16 * wg + 2 * q + (odd ? 1 : 0);
+            *reinterpret_cast<uint32_t*>(sm + SM_OSTG + sw128_offset(64, t, i & ~1)) =
+                odd ? pack_bf16(recv, o1) : pack_bf16(o0, recv);
+          }
         } else {
           // the sequence's last, partial chunk: plain stores of the valid rows
           const int64_t ostride = (p.layout == KDA_LAYOUT_BNSD) ? kD : (int64_t)p.Nv * kD;
           __nv_bfloat16* orow = p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t0) + i;
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int t = wg * 32 + 16 * ch + e;
-              if (t < n) orow[t * ostride] = __float2bfloat16_rn(__uint_as_float(vo[ch][e]));
-            }
+          for (int e = 0; e < 16; ++e) {
+            const int t = 16 * wg + e;
+            if (t < n) orow[t * ostride] = __float2bfloat16_rn(__uint_as_float(vo[e]));
+          }
         }
         KDA_TS(18);
+        uint32_t v0[16], v1[16], hi[16], lo[16];
+        const int col = wg * 32;
+        tmem_ld16(tl + TC_S + col, v0);
+        tmem_ld16(tl + TC_S + col + 16, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t v0[16], v1[16], pk[16];
-          const int col = wg * 64 + 32 * ch;
-          tmem_ld16(tbase + wlane + TC_S + col, v0);
-          tmem_ld16(tbase + wlane + TC_S + col + 16, v1);
-          tmem_wait_ld();
+        for (int e = 0; e < 8; ++e) {
+          const float a0 = __uint_as_float(v0[2 * e]), a1 = __uint_as_float(v0[2 * e + 1]);
+          const float c0 = __uint_as_float(v1[2 * e]), c1 = __uint_as_float(v1[2 * e + 1]);
+          hi[e] = pack_bf16(a0, a1);
+          hi[8 + e] = pack_bf16(c0, c1);
+          lo[e] = pack_bf16(a0 - bf16_round(a0), a1 - bf16_round(a1));
+          lo[8 + e] = pack_bf16(c0 - bf16_round(c0), c1 - bf16_round(c1));
+        }
+        tmem_st16(tl + TC_SHI + col / 2, hi);
+        tmem_st16(tl + TC_SLO + col / 2, lo);
+        if (last) {
+          float* dst = p.Sf + sbase_g + (size_t)i * kD + col;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            pk[e] = pack_bf16(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
-            pk[8 + e] = pack_bf16(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]));
-          }
-          tmem_st16(tbase + wlane + TC_S0 + col / 2, pk);
-          if (last) {
-            float* dst = p.Sf + sbase_g + (size_t)i * kD + col;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-              *reinterpret_cast<float4*>(dst + e) = make_float4(
-                  __uint_as_float(v0[e]), __uint_as_float(v0[e + 1]), __uint_as_float(v0[e + 2]),
-                  __uint_as_float(v0[e + 3]));
-              *reinterpret_cast<float4*>(dst + 16 + e) = make_float4(
-                  __uint_as_float(v1[e]), __uint_as_float(v1[e + 1]), __uint_as_float(v1[e + 2]),
-                  __uint_as_float(v1[e + 3]));
-            }
+          for (int e = 0; e < 16; e += 4) {
+            *reinterpret_cast<float4*>(dst + e) = make_float4(
+                __uint_as_float(v0[e]), __uint_as_float(v0[e + 1]), __uint_as_float(v0[e + 2]),
+                __uint_as_float(v0[e + 3]));
+            *reinterpret_cast<float4*>(dst + 16 + e) = make_float4(
+                __uint_as_float(v1[e]), __uint_as_float(v1[e + 1]), __uint_as_float(v1[e + 2]),
+                __uint_as_float(v1[e + 3]));
           }
         }
         tmem_wait_st();
@@ -909,17 +1046,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncthreads();
       KDA_TS(10);
-      if (tid == 0 && n == kChunk) {
-        int oc1, oc2;
-        if (p.layout == KDA_LAYOUT_BNSD) {
-          oc1 = t0;
-          oc2 = b * p.Nv + h;
-        } else {
-          oc1 = h;
-          oc2 = (p.layout == KDA_LAYOUT_BSND ? b * p.S : tok0) + t0;
-        }
-        tma_store_3d(&maps.o, sbase + SM_OSTG, 0, oc1, oc2);
-        tma_store_3d(&maps.o, sbase + SM_OSTG + 8192, 64, oc1, oc2);
+      if (st_thread && n == kChunk) {
+        int qc1, qc2, oc1, oc2;
+        const UnitRec ur{b, h, 0, tok0, nch};
+        chunk_coords(p, ur, c, qc1, qc2, oc1, oc2);
+        const int half = warp - 9;
+        tma_store_3d(&maps.o, sbase + SM_OSTG + half * 8192, 64 * half, oc1, oc2);
         tma_store_commit();
       }
       if (*abort_flag) {
@@ -938,9 +1070,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // drain: loads still in flight must land, and stores complete, before this CTA exits
+  if (st_thread) tma_store_wait_all();
   if (tid == 0) {
-    tma_store_wait_all();
-    while (gidx < issued) {
+    while (gidx < prod->issued) {
       if (!mbar_wait_bounded(sbase + SM_BAR + 8u * (gidx & 1), (gidx >> 1) & 1u, kWaitLimit)) {
         atomicExch(p.status, DS_TIMEOUT);
         break;
