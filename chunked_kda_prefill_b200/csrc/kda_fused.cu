@@ -121,6 +121,10 @@ __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
 // the two floats of a packed bf16 pair (low half = first element)
 __device__ __forceinline__ float bf16_lo_of(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_of(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// bf16 hi part of (a, b) packed, and the packed bf16 of the remainders (a, b) - hi
+__device__ __forceinline__ uint32_t split_lo(float a, float b, uint32_t hi) {
+  return pack_bf16(a - bf16_lo_of(hi), b - bf16_hi_of(hi));
+}
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
@@ -327,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) {
           const float x0 = __uint_as_float(fv[2 * c]), x1 = __uint_as_float(fv[2 * c + 1]);
           hi[c] = pack_bf16(x0, x1);
-          lo[c] = pack_bf16(x0 - bf16_round(x0), x1 - bf16_round(x1));
+          lo[c] = split_lo(x0, x1, hi[c]);
         }
         tmem_st16(tl + TC_S + col0, fv);
         tmem_st8(tl + TC_SHI + col0 / 2, hi);
@@ -435,8 +439,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float qv[4], kv[4];
-          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r0 + i, j0)), qv);
-          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r0 + i, j0)), kv);
+          const bool valid = r0 + i < n;
+          const uint2 zero2 = make_uint2(0u, 0u);
+          const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r0 + i, j0));
+          const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r0 + i, j0));
+          unpack4(valid ? qw : zero2, qv);
+          unpack4(valid ? kw : zero2, kv);
           float ssq = 0.f, ssk = 0.f;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -457,17 +465,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const int r = r0 + i;
           const bool valid = r < n;
+          // rows past the valid length (whatever the storage holds there) become exact zeros
+          const uint2 zero2 = make_uint2(0u, 0u);
+          const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j0));
+          const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0));
           float qv[4], kv[4];
-          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j0)), qv);
-          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0)), kv);
+          unpack4(valid ? qw : zero2, qv);
+          unpack4(valid ? kw : zero2, kv);
           const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
           const float rk = rsqrtf(rkv[i] + 1e-6f);
-          float ka[4], qa[4], kt[4], qt[4], kh[4], khl[4], b0[4], b1[4], b2[4], b3[4];
+          float ka[4], qa[4], kt[4], qt[4], kh[4], b0[4], b1[4], b2[4], b3[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float Gv = G[i][e];
-            const float kn = valid ? kv[e] * rk : 0.f;
-            const float qn = valid ? qv[e] * rq : 0.f;
+            const float kn = kv[e] * rk;
+            const float qn = qv[e] * rq;
             const float fA = ex2(Gv - k4[CST_REF][e]);
             const float kbe = kn * ex2(k4[CST_GE][e] - Gv);
             ka[e] = kn * fA;
@@ -475,17 +487,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             kt[e] = ka[e] * k4[CST_P2REF][e];
             qt[e] = qa[e] * k4[CST_P2REF][e];
             kh[e] = kbe * k4[CST_KFAC][e];
-            khl[e] = kh[e] - bf16_round(kh[e]);
             b0[e] = kbe * k4[CST_CDIAG][e];  // B^(Jb): diagonal block
             b1[e] = kbe;                     // B^(Jb+1): reference row is this block's last row
             b2[e] = kbe * k4[CST_C2][e];     // B^(Jb+2)
             b3[e] = kbe * k4[CST_C3][e];     // B^(Jb+3)
           }
+          const uint2 khp = pack4(kh[0], kh[1], kh[2], kh[3]);
+          khlo[i] = make_uint2(split_lo(kh[0], kh[1], khp.x), split_lo(kh[2], kh[3], khp.y));
           *reinterpret_cast<uint2*>(sm + SM_AOP + sw128_offset(128, r, j0)) = pack4(ka[0], ka[1], ka[2], ka[3]);
           *reinterpret_cast<uint2*>(sm + SM_AOP + sw128_offset(128, 64 + r, j0)) = pack4(qa[0], qa[1], qa[2], qa[3]);
           *reinterpret_cast<uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j0)) = pack4(qt[0], qt[1], qt[2], qt[3]);
-          *reinterpret_cast<uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0)) = pack4(kh[0], kh[1], kh[2], kh[3]);
-          khlo[i] = pack4(khl[0], khl[1], khl[2], khl[3]);
+          *reinterpret_cast<uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0)) = khp;
           *reinterpret_cast<uint2*>(sq + OFF_G + atom_off(QGV_ATOM, r, j0)) = pack4(kt[0], kt[1], kt[2], kt[3]);
           *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb) + r, j0)) =
               pack4(b0[0], b0[1], b0[2], b0[3]);
@@ -795,14 +807,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 bb = *reinterpret_cast<const float4*>(beta_s + s0 + 4);
         const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
         const float bv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
-        float f[8], fl[8];
+        float f[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          f[e] = (s0 + e <= r) ? xv[e] * bv[e] : 0.f;
-          fl[e] = f[e] - bf16_round(f[e]);
-        }
-        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, r, s0)) = pack8(f);
-        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, 64 + r, s0)) = pack8(fl);
+        for (int e = 0; e < 8; ++e) f[e] = (s0 + e <= r) ? xv[e] * bv[e] : 0.f;
+        const uint4 hi = pack8(f);
+        const uint4 lo = make_uint4(split_lo(f[0], f[1], hi.x), split_lo(f[2], f[3], hi.y),
+                                    split_lo(f[4], f[5], hi.z), split_lo(f[6], f[7], hi.w));
+        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, r, s0)) = hi;
+        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, 64 + r, s0)) = lo;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -949,7 +961,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float d1 = __uint_as_float(vu[2 * e + 1]) + __uint_as_float(va[2 * e + 1]) +
                            __uint_as_float(vb[2 * e + 1]);
           hi[e] = pack_bf16(d0, d1);
-          lo[e] = pack_bf16(d0 - bf16_round(d0), d1 - bf16_round(d1));
+          lo[e] = split_lo(d0, d1, hi[e]);
         }
         tmem_st8(tl + TC_DHI + 8 * wg, hi);
         tmem_st8(tl + TC_DLO + 8 * wg, lo);
@@ -1023,8 +1035,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float c0 = __uint_as_float(v1[2 * e]), c1 = __uint_as_float(v1[2 * e + 1]);
           hi[e] = pack_bf16(a0, a1);
           hi[8 + e] = pack_bf16(c0, c1);
-          lo[e] = pack_bf16(a0 - bf16_round(a0), a1 - bf16_round(a1));
-          lo[8 + e] = pack_bf16(c0 - bf16_round(c0), c1 - bf16_round(c1));
+          lo[e] = split_lo(a0, a1, hi[e]);
+          lo[8 + e] = split_lo(c0, c1, hi[8 + e]);
         }
         tmem_st16(tl + TC_SHI + col / 2, hi);
         tmem_st16(tl + TC_SLO + col / 2, lo);
