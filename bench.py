@@ -251,9 +251,7 @@ def run_ours(args, rank, world):
         if dist is not None:
             dist.barrier()
 
-    w = W.workload(args.workload)
-    if world > 1:
-        w.seed = w.seed + 1000 * rank
+    w = rank_workload(args.workload, rank, world)
     inp = W.generate(w)
     host = {}
     for n in ("q", "k", "v", "g", "beta"):
@@ -337,11 +335,11 @@ def run_ours(args, rank, world):
         torch.cuda.synchronize(dev)
         barrier()
         e_ms = _max_over_ranks(e0.elapsed_time(e1), dist, dev)
-        e2e = {"value": world * w.token_heads * steps_e2e / (e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": job_throughput(w.token_heads, world, steps_e2e, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": steps_e2e}
 
-    value = world * w.token_heads * args.steps / (elapsed_ms / 1e3)
+    value = job_throughput(w.token_heads, world, args.steps, elapsed_ms)
     peak, peak_kind = measured_peaks()
     abytes = algorithmic_bytes(w, True)
     achieved = abytes / (kernel_ms / 1e3) / 1e9
@@ -364,6 +362,20 @@ def run_ours(args, rank, world):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def rank_workload(idx: int, rank: int, world: int) -> W.Workload:
+    """The workload replica of one rank: same shapes, its own seed (rank r adds 1000 r)."""
+    w = W.workload(idx)
+    if world > 1:
+        w.seed = w.seed + 1000 * rank
+    return w
+
+
+def job_throughput(token_heads: int, world: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job token-heads/s: every rank processes `token_heads` per step; the time is the
+    slowest rank's (max over ranks)."""
+    return world * token_heads * steps / (elapsed_ms / 1e3)
 
 
 def _max_over_ranks(x, dist, dev):

@@ -27,6 +27,7 @@ enum : int {
   ST_TS_MN = 5,    // A from TMEM, B MN-major
   ST_TF32_SS = 6,  // kind::tf32, A K-major fp32, B K-major fp32 (shared memory)
   ST_TF32_TS = 7,  // kind::tf32, A fp32 from TMEM, B K-major fp32
+  ST_TIMEOUT = 8,  // bounded wait on a barrier that nothing arrives on: must give up and report
 };
 
 constexpr uint32_t kWaitLimit = 1u << 24;
@@ -47,6 +48,7 @@ __global__ void __launch_bounds__(128, 1)
 
   if (tid == 0) {
     mbar_init(bar_a, 1);
+    mbar_init(bar_a + 8, 1);  // ST_TIMEOUT's barrier: no thread, MMA or copy ever arrives on it
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -58,7 +60,10 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tbase = *tslot;
 
-  if (variant == ST_TF32_SS || variant == ST_TF32_TS) {
+  if (variant == ST_TIMEOUT) {
+    // a short bounded wait that must run out; the kernel then leaves through its normal exit
+    if (tid == 0 && !mbar_wait_bounded(bar_a + 8, 0, 1u << 14)) atomicExch(err, 3);
+  } else if (variant == ST_TF32_SS || variant == ST_TF32_TS) {
     // fp32 operands (tf32 MMA): A [128][K] (fp32, passed as A), B [N][K] (fp32), both K-major
     const float* Af = reinterpret_cast<const float*>(A);
     const float* Bf = reinterpret_cast<const float*>(B);
@@ -196,10 +201,10 @@ extern "C" __attribute__((visibility("default"))) int kda_selftest(
     int variant, const void* A, const void* B, float* D, int N, int K, void* raw,
     const void* tma_src, int tma_rows, int row0, int* err_dev, void* stream) {
   using namespace kda;
-  if (variant < 0 || variant > ST_TF32_TS) return 1;
-  if (variant != ST_TMA && (!A || !B || !D || N < 16 || N > 128 || N % 16 != 0)) return 1;
+  if (variant < 0 || variant > ST_TIMEOUT) return 1;
+  if (variant != ST_TMA && variant != ST_TIMEOUT && (!A || !B || !D || N < 16 || N > 128 || N % 16 != 0)) return 1;
   if (variant != ST_TMA && variant < ST_TF32_SS && K != 64 && K != 128) return 1;
-  if (variant >= ST_TF32_SS && K != 32 && K != 64) return 1;
+  if ((variant == ST_TF32_SS || variant == ST_TF32_TS) && K != 32 && K != 64) return 1;
   if ((variant == ST_SS_KMN || variant == ST_TS_MN) && N != 64 && N != 128) return 1;
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));

@@ -93,3 +93,34 @@ def test_tf32_mma_plumbing(variant, N, K, cuda_ok):
     ref = A.double() @ B.double().t()
     got = D.cpu().double()
     assert torch.allclose(got, ref, rtol=1e-5, atol=1e-4), (got - ref).abs().max()
+
+
+def test_bounded_wait_gives_up_and_the_context_survives(cuda_ok):
+    """Failure detection without a fault: a bounded mbarrier wait on a barrier that nothing
+    arrives on must run out, report it through the status word, and leave the context usable."""
+    f = _lib()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert f(8, None, None, None, 0, 0, None, None, 0, 0, err.data_ptr(), s) == 3
+    assert int(err.item()) == 3
+    # the same context still runs a normal MMA case correctly
+    g = torch.Generator().manual_seed(5)
+    A = torch.randn(128, 64, generator=g).to(torch.bfloat16)
+    B = torch.randn(64, 64, generator=g).to(torch.bfloat16)
+    D = torch.full((128, 64), float("nan"), dtype=torch.float32, device="cuda")
+    assert f(0, A.cuda().data_ptr(), B.cuda().data_ptr(), D.data_ptr(), 64, 64, None, None, 0, 0,
+             err.data_ptr(), s) == 0
+    ref = A.double() @ B.double().t()
+    assert torch.allclose(D.cpu().double(), ref, rtol=1e-5, atol=1e-4)
+
+
+def test_device_timeout_word_maps_to_status_code(cuda_ok):
+    """A kernel that gave up a bounded wait leaves DS_TIMEOUT (2) in the workspace status word;
+    kda_device_status reports it as KDA_ERR_TIMEOUT, and a plan mismatch (1) as KDA_ERR_PLAN."""
+    ws = torch.zeros(64, dtype=torch.int32, device="cuda")
+    kda.device_status(ws)  # 0: fine
+    for word, name in ((2, "KDA_ERR_TIMEOUT"), (1, "KDA_ERR_PLAN")):
+        ws[0] = word
+        with pytest.raises(kda.KdaError) as e:
+            kda.device_status(ws)
+        assert e.value.name == name
