@@ -5,6 +5,6 @@ the thin Python binding over it.  Build the library with
 ``python -m chunked_kda_prefill_b200.build``.
 """
 from ._lib import EXPORTS, LIB_PATH, KdaError, KdaShape, load  # noqa: F401
-from .api import (KdaPlan, LAYOUTS, device_status, flash_kda, flash_kda_noalloc,  # noqa: F401
+from .api import (KdaPlan, LAYOUTS, decode, device_status, flash_kda, flash_kda_noalloc,  # noqa: F401
                   forward_kernel_names,
                   kernels_per_forward, make_plan, plan)

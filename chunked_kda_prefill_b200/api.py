@@ -180,6 +180,43 @@ def flash_kda_noalloc(q, k, v, g, beta, scale: float, initial_state, A_log, dt_b
     return out, final_state
 
 
+def decode(q, k, v, g, beta, scale: float, state, A_log, dt_bias, lower_bound: float,
+           out: torch.Tensor | None = None, state_out: torch.Tensor | None = None,
+           stream: torch.cuda.Stream | None = None):
+    """One decode step (one token per sequence) through kda_decode.
+
+    q, k: bf16 [B, Nqk, 128]; v, g: bf16 [B, Nv, 128]; beta: bf16 [B, Nv]; state: fp32
+    [B, Nv, 128, 128] or None (zeros).  Returns (out [B, Nv, 128] bf16, state_out); pass
+    ``state_out=state`` to update the state in place.
+    """
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("decode runs on a CUDA device only")
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta")):
+        _expect(t, name, torch.bfloat16, dev)
+    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias")):
+        _expect(t, name, torch.float32, dev)
+    if state is not None:
+        _expect(state, "state", torch.float32, dev)
+    if q.dim() != 3 or v.dim() != 3 or beta.shape != v.shape[:2]:
+        raise KdaError(3, "decode expects q/k [B,Nqk,D], v/g [B,Nv,D], beta [B,Nv]")
+    B, Nqk, D = q.shape
+    Nv = v.shape[1]
+    if out is None:
+        out = torch.empty_like(v)
+    if state_out is None:
+        state_out = torch.empty((B, Nv, D, D), dtype=torch.float32, device=dev)
+    _expect(out, "out", torch.bfloat16, dev)
+    _expect(state_out, "state_out", torch.float32, dev)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    code = _lib.load().kda_decode(B, Nqk, Nv, D, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                  g.data_ptr(), beta.data_ptr(), float(scale), _ptr(state),
+                                  A_log.data_ptr(), dt_bias.data_ptr(), float(lower_bound),
+                                  out.data_ptr(), state_out.data_ptr(), s.cuda_stream)
+    check(code, "kda_decode")
+    return out, state_out
+
+
 def device_status(workspace: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
     """Synchronise and raise if the last forward on this workspace recorded a device error."""
     s = stream if stream is not None else torch.cuda.current_stream(workspace.device)

@@ -164,6 +164,30 @@ KDA_API kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int32_t
                                          const float* dt_bias, float lower_bound, void* out,
                                          float* final_state, kda_stream_t stream);
 
+/* The single-token decode step that follows a prefill: one step of the recurrence the chunked
+ * forward computes in 64-token blocks (FlashKDA README, 功能说明; FLA PR 656, "[kda] add
+ * recursive block intra", keeps the same recurrence as its naive token-by-token kernel):
+ *     S <- S Diag(e^g);  S <- S + beta (v - S k^) k^T;  o = scale S q^
+ * with kda_forward's in-op activations (q, k L2-normalised; beta = sigmoid(logit);
+ * g = lower_bound * sigmoid(e^A_log[h] (g_raw + dt_bias[h,:]))), one token per sequence.
+ *   B, Nqk, Nv, D: sequences, query/key heads, value heads (Nv % Nqk == 0; value head h reads
+ *                  query/key head h / (Nv / Nqk)), head dim (must be 128).
+ *   q, k         : bf16 [B, Nqk, D];  v, g: bf16 [B, Nv, D];  beta: bf16 [B, Nv] (logits).
+ *   scale        : finite;  A_log: fp32 [Nv];  dt_bias: fp32 [Nv, D];  lower_bound in [-5, 0].
+ *   state_in     : fp32 [B, Nv, D(Dv), D(Dk)], or NULL for zeros.
+ *   state_out    : fp32 [B, Nv, D, D]; may be state_in itself (the update is done in place, each
+ *                  state row read before it is written) but must not overlap it otherwise.
+ *   out          : bf16 [B, Nv, D], rounded to nearest even.
+ * The caller owns every buffer; the call allocates nothing.  Pointers are device memory, 16-byte
+ * aligned (beta 2-byte).  Errors: KDA_ERR_DIM, _SHAPE, _HEADS, _NULL, _LOWER_BOUND (also a
+ * non-finite scale), _ALIGN, _ALIAS (an output overlapping an input or the other output),
+ * _DEVICE (not sm_100), _CUDA (launch failure).  Asynchronous on `stream`. */
+KDA_API kda_status_t kda_decode(int32_t B, int32_t Nqk, int32_t Nv, int32_t D, const void* q,
+                                const void* k, const void* v, const void* g, const void* beta,
+                                float scale, const float* state_in, const float* A_log,
+                                const float* dt_bias, float lower_bound, void* out,
+                                float* state_out, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -152,3 +152,31 @@ def test_status_strings(L):
     for code in range(16):
         s = L.kda_status_string(code).decode()
         assert s.startswith("KDA_")
+
+
+def _dec(L, B=2, Nqk=1, Nv=2, D=128, **kw):
+    a = dict(q=0x10000000, k=0x11000000, v=0x12000000, g=0x13000000, beta=0x14000000, scale=0.09,
+             s0=0x20000000, A_log=0x15000000, dt=0x16000000, lb=-5.0, out=0x17000000,
+             s1=0x30000000)
+    a.update(kw)
+    return L.kda_decode(B, Nqk, Nv, D, a["q"], a["k"], a["v"], a["g"], a["beta"], a["scale"],
+                        a["s0"], a["A_log"], a["dt"], a["lb"], a["out"], a["s1"], None)
+
+
+def test_decode_argument_checks(L):
+    assert _dec(L, D=64) == 5
+    assert _dec(L, B=0) == 3
+    assert _dec(L, Nv=3, Nqk=2) == 4
+    assert _dec(L, q=None) == 1
+    assert _dec(L, s1=None) == 1
+    assert _dec(L, lb=0.25) == 6
+    assert _dec(L, scale=float("nan")) == 6
+    assert _dec(L, v=0x12000008) == 14                  # v not 16-byte aligned
+    assert _dec(L, beta=0x14000001) == 14               # beta not 2-byte aligned
+    assert _dec(L, s1=0x20000000 + 4096) == 9           # state_out partly overlaps state_in
+    assert _dec(L, out=0x12000000 + 256) == 9           # out overlaps v
+    assert _dec(L, out=0x30000000 + 4096) == 9          # out overlaps state_out
+    # in place (state_out == state_in) and a zero initial state are allowed: the remaining
+    # checks need a GPU (none here -> CUDA/device error)
+    assert _dec(L, s1=0x20000000) in (11, 13)
+    assert _dec(L, s0=None) in (11, 13)
