@@ -348,7 +348,7 @@ def run_ours(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 inputs, random-init A_log/dt_bias)",
             "config": _config(w, world), "clocks": clk.report(), "e2e": e2e,
-            "gpu_launches": args.steps * kda.kernels_per_forward(),
+            "gpu_launches": args.steps * kda.kernels_per_forward(plan),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": ncu_traffic(w.name),
                          "kernel": kda.forward_kernel_names(),

@@ -9,7 +9,8 @@ LIB_PATH = os.path.join(PKG, "libkda.so")
 
 # Every symbol include/kda.h declares.
 EXPORTS = ("kda_status_string", "kda_plan_size", "kda_plan", "kda_workspace_size",
-           "kda_forward", "kda_device_status", "kda_forward_noalloc", "kda_decode")
+           "kda_forward", "kda_device_status", "kda_forward_noalloc", "kda_decode",
+           "kda_plan_segmented")
 
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_NULL", 2: "KDA_ERR_LAYOUT", 3: "KDA_ERR_SHAPE",
           4: "KDA_ERR_HEADS", 5: "KDA_ERR_DIM", 6: "KDA_ERR_LOWER_BOUND", 7: "KDA_ERR_SEQLENS",
@@ -57,10 +58,11 @@ def load():
     L.kda_device_status.argtypes = [vp, vp]
     L.kda_forward_noalloc.argtypes = [p_shape, p_i32, vp, sz, vp, vp, vp, vp, vp, ctypes.c_float,
                                       vp, vp, vp, ctypes.c_float, vp, vp, vp]
+    L.kda_plan_segmented.argtypes = [p_shape, p_i32, i32, i32, p_i32, sz]
     L.kda_decode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
                              ctypes.c_float, vp, vp, vp]
     for f in ("kda_plan_size", "kda_plan", "kda_workspace_size", "kda_forward",
-              "kda_device_status", "kda_forward_noalloc", "kda_decode"):
+              "kda_device_status", "kda_forward_noalloc", "kda_decode", "kda_plan_segmented"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L

@@ -40,6 +40,11 @@ class KdaPlan:
     def total_chunks(self) -> int:
         return int(self.host[11])
 
+    @property
+    def segment_chunks(self) -> int:
+        """Segment length of a chunk-parallel (segmented) schedule; 0 when units run whole."""
+        return int(self.host[14])
+
     def workspace(self) -> torch.Tensor:
         """A workspace owned by the plan, allocated on first use and reused afterwards."""
         if self._workspace is None or self._workspace.device != self.dev.device:
@@ -67,8 +72,12 @@ def _shape_from(q: torch.Tensor, v: torch.Tensor, layout: str, cu_seqlens) -> Kd
 
 
 def make_plan(shape: KdaShape, layout: str, cu_seqlens=None, num_sms: int | None = None,
-              device=None) -> KdaPlan:
-    """Build a plan from an explicit shape (host work only, plus one small device copy)."""
+              device=None, segment_chunks: int | None = None) -> KdaPlan:
+    """Build a plan from an explicit shape (host work only, plus one small device copy).
+
+    ``segment_chunks``: None picks the schedule (kda_plan); 0 runs every unit whole; n > 0 cuts
+    units into segments of n chunks (kda_plan_segmented).
+    """
     L = _lib.load()
     n = ctypes.c_size_t(0)
     check(L.kda_plan_size(ctypes.byref(shape), ctypes.byref(n)), "kda_plan_size")
@@ -81,8 +90,12 @@ def make_plan(shape: KdaShape, layout: str, cu_seqlens=None, num_sms: int | None
     if num_sms is None:
         num_sms = (torch.cuda.get_device_properties(device).multi_processor_count
                    if torch.cuda.is_available() else 148)
-    check(L.kda_plan(ctypes.byref(shape), cu_ptr, int(num_sms),
-                     host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), host.size), "kda_plan")
+    hp = host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    if segment_chunks is None:
+        check(L.kda_plan(ctypes.byref(shape), cu_ptr, int(num_sms), hp, host.size), "kda_plan")
+    else:
+        check(L.kda_plan_segmented(ctypes.byref(shape), cu_ptr, int(num_sms), int(segment_chunks),
+                                   hp, host.size), "kda_plan_segmented")
     ws = ctypes.c_size_t(0)
     check(L.kda_workspace_size(host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), host.size,
                                ctypes.byref(ws)), "kda_workspace_size")
@@ -94,14 +107,16 @@ def make_plan(shape: KdaShape, layout: str, cu_seqlens=None, num_sms: int | None
 
 
 def plan(q: torch.Tensor, v: torch.Tensor, initial_state: torch.Tensor | None, layout: str,
-         cu_seqlens=None, num_sms: int | None = None) -> KdaPlan:
+         cu_seqlens=None, num_sms: int | None = None,
+         segment_chunks: int | None = None) -> KdaPlan:
     """flash_kda_metadata counterpart: shapes, layout and valid lengths -> schedule."""
     if isinstance(cu_seqlens, torch.Tensor):
         cu_seqlens = cu_seqlens.detach().to("cpu").numpy()
     shape = _shape_from(q, v, layout, cu_seqlens)
     if initial_state is not None and initial_state.shape[0] != shape.B:
         raise KdaError(3, "initial_state batch does not match the number of sequences")
-    return make_plan(shape, layout, cu_seqlens, num_sms, device=q.device)
+    return make_plan(shape, layout, cu_seqlens, num_sms, device=q.device,
+                     segment_chunks=segment_chunks)
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -223,9 +238,9 @@ def device_status(workspace: torch.Tensor, stream: torch.cuda.Stream | None = No
     check(_lib.load().kda_device_status(workspace.data_ptr(), s.cuda_stream), "kda_device_status")
 
 
-def kernels_per_forward() -> int:
-    """Kernels of this library that one kda_forward launches."""
-    return 1
+def kernels_per_forward(plan: KdaPlan | None = None) -> int:
+    """Kernels of this library that one kda_forward launches (three under a segmented plan)."""
+    return 3 if plan is not None and plan.segment_chunks > 0 else 1
 
 
 def forward_kernel_names() -> str:

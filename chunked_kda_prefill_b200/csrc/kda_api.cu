@@ -1,6 +1,7 @@
 // kda_api.cu -- kda_forward / kda_device_status: argument checks, then the kernel launches.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdint>
 
@@ -63,7 +64,8 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
       if (reinterpret_cast<uintptr_t>(ptr) & 15u) return KDA_ERR_ALIGN;
     if (reinterpret_cast<uintptr_t>(beta) & 1u) return KDA_ERR_ALIGN;
   }
-  const size_t need = (path == PATH_SIMT) ? simt_workspace_bytes(plan_host) : kWsHeaderBytes;
+  const size_t need =
+      (path == PATH_SIMT) ? simt_workspace_bytes(plan_host) : fused_workspace_bytes(plan_host);
   if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return KDA_ERR_WORKSPACE;
 
@@ -113,9 +115,31 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   p.Sf = final_state;
   p.tprof = tprof;
 
+  p.seg_chunks = plan_host[PH_SEG_CHUNKS];
+  p.states = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeaderBytes);
+
   if (cudaMemsetAsync(workspace, 0, 4, stream) != cudaSuccess) return KDA_ERR_CUDA;
-  const cudaError_t e = (path == PATH_SIMT) ? launch_simt(p, plan_host[PH_TOTAL_CHUNKS], stream)
-                                            : launch_fused(p, dbg, stream);
+  cudaError_t e;
+  if (path == PATH_SIMT) {
+    e = launch_simt(p, plan_host[PH_TOTAL_CHUNKS], stream);
+  } else if (p.seg_chunks <= 0) {
+    p.mode = 0;
+    p.n_items = p.n_units;
+    e = launch_fused(p, dbg, stream);
+  } else {
+    // segmented schedule: segment summaries, start states, outputs
+    const SegCounts sc = seg_counts(plan_host);
+    if (sc.items_a > INT_MAX) return KDA_ERR_SHAPE;
+    p.mode = 1;
+    p.n_items = (int)sc.items_a;
+    e = launch_fused(p, dbg, stream);
+    if (e == cudaSuccess) e = launch_combine(p, stream);
+    if (e == cudaSuccess && sc.items_c > 0) {
+      p.mode = 2;
+      p.n_items = (int)sc.items_c;
+      e = launch_fused(p, dbg, stream);
+    }
+  }
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -134,37 +134,125 @@ struct Maps {
   CUtensorMap q, k, v, g, o;
 };
 
-// A unit's plan record as the producer keeps it.
-struct UnitRec {
-  int b, h, hq, tok0, nch;
+// A work item: a range of chunks of one (sequence, value head) unit, the state it starts from
+// and where its final state goes.  Mode 0 runs units whole.  Under a segmented plan, mode 1 runs
+// per unit its first segment from the true initial state (outputs written) and, for every later
+// segment s, an R run (from S = 0) and an M run (from S = I with v = 0) that leave the segment's
+// affine map S -> S M_s + R_s in state slot s; mode 2 runs every later segment from its start
+// state (computed in between by the combine kernel), writing outputs and the final state.
+struct Item {
+  int b, h, hq, tok0, L;  // the sequence, its first packed row and its length
+  int c_begin, c_end;     // chunks of the sequence this item runs
+  int coff;               // the unit's chunk offset (debug dump)
+  int ident;              // start from the identity (M run)
+  const float* s_in;      // start state (null: zero; ignored for the identity)
+  float* s_out;           // where the final state goes (null: nowhere)
+  int write_out, zero_v, pad;  // write outputs; treat v as zero; zero-fill rows past L
 };
-// The load schedule, kept in shared memory: the cursor (next (unit, chunk) of this CTA's stream,
-// chunks planned so far, the plan records of the current and next unit, read one unit ahead so
-// no global load sits on the issue path), written by thread 0 only; and the chunk whose tiles
-// go out during the current chunk, which ten warps read to issue one TMA box each.
-struct Producer {
-  int pu, pc;
-  uint32_t issued;
-  UnitRec cur, next;
-  int ld_valid, ld_c, ld_slot;
-  UnitRec ld_rec;
+
+__device__ __forceinline__ float* slot_ptr(const Params& p, int slot, int part) {
+  return p.states + (size_t)slot * kSlotFloats + (size_t)part * kD * kD;
+}
+
+// Item i of this launch (every argument comes from the plan; see the Item comment).
+__device__ Item item_of(const Params& p, int i) {
+  const int32_t* R = p.plan + kPlanHeader;
+  int u = i;
+  if (p.mode != 0) {  // the unit whose item range holds i (item offsets increase along the plan)
+    int lo = 0, hi = p.n_units - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      const int base = R[mid * kPlanRecord + PR_SEG_BASE];
+      const int off = (p.mode == 1) ? mid + 2 * base : base;
+      if (off <= i) lo = mid; else hi = mid - 1;
+    }
+    u = lo;
+  }
+  const int32_t* rec = R + u * kPlanRecord;
+  Item it;
+  it.b = rec[PR_B];
+  it.h = rec[PR_H];
+  it.hq = rec[PR_HQ];
+  it.tok0 = rec[PR_TOK_START];
+  it.L = rec[PR_LEN];
+  it.coff = rec[PR_CHUNK_OFFSET];
+  const int nch = rec[PR_CHUNKS];
+  const size_t bh = ((size_t)it.b * p.Nv + it.h) * kD * kD;
+  const float* s0 = p.S0 ? p.S0 + bh : nullptr;
+  it.ident = 0;
+  it.zero_v = 0;
+  if (p.mode == 0) {
+    it.c_begin = 0;
+    it.c_end = nch;
+    it.s_in = s0;
+    it.s_out = p.Sf + bh;
+    it.write_out = 1;
+    it.pad = 1;
+    return it;
+  }
+  const int seg = p.seg_chunks, nseg = (nch + seg - 1) / seg;
+  const int base = rec[PR_SEG_BASE];
+  int sgm;
+  if (p.mode == 1) {
+    const int j = i - (u + 2 * base);
+    sgm = (j + 1) >> 1;
+    if (j == 0) {  // the first segment, from the true initial state
+      it.s_in = s0;
+      it.s_out = (nseg == 1) ? p.Sf + bh : slot_ptr(p, base, SLOT_START);
+      it.write_out = 1;
+      it.pad = (nseg == 1);
+    } else {
+      it.s_in = nullptr;
+      it.write_out = 0;
+      it.pad = 0;
+      if (j & 1) {
+        it.s_out = slot_ptr(p, base + sgm - 1, SLOT_R);
+      } else {
+        it.ident = 1;
+        it.zero_v = 1;
+        it.s_out = slot_ptr(p, base + sgm - 1, SLOT_M);
+      }
+    }
+  } else {
+    sgm = i - base + 1;
+    it.s_in = slot_ptr(p, base + sgm - 1, SLOT_START);
+    it.s_out = (sgm == nseg - 1) ? p.Sf + bh : nullptr;
+    it.write_out = 1;
+    it.pad = (sgm == nseg - 1);
+  }
+  it.c_begin = sgm * seg;
+  it.c_end = min(nch, it.c_begin + seg);
+  return it;
+}
+
+// The part of an item the TMA producer needs.
+struct LoadRec {
+  int b, h, hq, tok0, c_begin, c_end;
 };
-static_assert(sizeof(Producer) <= SM_END - SM_PROD, "producer state overflows its region");
-__device__ __forceinline__ UnitRec read_rec(const Params& p, int u) {
-  UnitRec r{0, 0, 0, 0, 0};
-  if (u < p.n_units) {
-    const int32_t* rec = p.plan + kPlanHeader + u * kPlanRecord;
-    r.b = rec[PR_B];
-    r.h = rec[PR_H];
-    r.hq = rec[PR_HQ];
-    r.tok0 = rec[PR_TOK_START];
-    r.nch = rec[PR_CHUNKS];
+__device__ __forceinline__ LoadRec load_rec(const Params& p, int i) {
+  LoadRec r{0, 0, 0, 0, 0, 0};
+  if (i < p.n_items) {
+    const Item it = item_of(p, i);
+    r = LoadRec{it.b, it.h, it.hq, it.tok0, it.c_begin, it.c_end};
   }
   return r;
 }
 
+// The load schedule, kept in shared memory: the cursor (next (item, chunk) of this CTA's stream,
+// chunks planned so far, the current and next item, read one item ahead so no global load sits
+// on the issue path), written by thread 0 only; and the chunk whose tiles go out during the
+// current chunk, which ten warps read to issue one TMA box each.
+struct Producer {
+  int pu, pc;
+  uint32_t issued;
+  LoadRec cur, next;
+  int ld_valid, ld_c, ld_slot;
+  LoadRec ld_rec;
+};
+static_assert(sizeof(Producer) <= SM_END - SM_PROD, "producer state overflows its region");
+
 // Tensor coordinates of chunk c of unit `ur` for the q/k maps (qc) and the v/g/out maps (vc).
-__device__ __forceinline__ void chunk_coords(const Params& p, const UnitRec& ur, int c, int& qc1,
+__device__ __forceinline__ void chunk_coords(const Params& p, const LoadRec& ur, int c, int& qc1,
                                              int& qc2, int& vc1, int& vc2) {
   const int t = c * kChunk;
   if (p.layout == KDA_LAYOUT_BNSD) {
@@ -179,7 +267,7 @@ __device__ __forceinline__ void chunk_coords(const Params& p, const UnitRec& ur,
 // 4-5 v, 6-7 k.  Every box arrives on the slot's barrier with its own byte count, so the eight
 // boxes can be issued by eight threads (a TMA issue occupies its thread for tens of cycles).
 __device__ __forceinline__ void issue_box(const Params& p, const Maps& m, uint32_t sbase,
-                                          const UnitRec& ur, int c, int slot, int box) {
+                                          const LoadRec& ur, int c, int slot, int box) {
   int qc1, qc2, vc1, vc2;
   chunk_coords(p, ur, c, qc1, qc2, vc1, vc2);
   const uint32_t bar = sbase + SM_BAR + 8u * slot;
@@ -245,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Producer* prod = reinterpret_cast<Producer*>(sm + SM_PROD);
   auto plan_load = [&]() {  // thread 0
     Producer& pr = *prod;
-    if (pr.pu >= p.n_units) {
+    if (pr.pu >= p.n_items) {
       pr.ld_valid = 0;
       return;
     }
@@ -254,11 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     pr.ld_c = pr.pc;
     pr.ld_slot = pr.issued & 1;
     ++pr.issued;
-    if (++pr.pc == pr.cur.nch) {
-      pr.pc = 0;
+    if (++pr.pc == pr.cur.c_end) {
       pr.pu += G_stride;
       pr.cur = pr.next;
-      pr.next = read_rec(p, pr.pu + G_stride);
+      pr.pc = pr.cur.c_begin;
+      pr.next = load_rec(p, pr.pu + G_stride);
     }
   };
   auto issue_planned = [&](int box) {
@@ -268,10 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool st_thread = lane == 0 && (warp == 9 || warp == 10);  // out-tile store issuers
   if (tid == 0) {
     prod->pu = blockIdx.x;
-    prod->pc = 0;
     prod->issued = 0;
-    prod->cur = read_rec(p, blockIdx.x);
-    prod->next = read_rec(p, blockIdx.x + G_stride);
+    prod->cur = load_rec(p, blockIdx.x);
+    prod->pc = prod->cur.c_begin;
+    prod->next = load_rec(p, blockIdx.x + G_stride);
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.k);
     tma_prefetch_desc(&maps.v);
@@ -300,18 +388,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   // phase-1 thread map: warp w owns rows 4w..4w+3 (16-row block w/4), lane owns columns 4l..4l+3
   const int r0 = 4 * warp, j0 = 4 * lane, Jb = warp >> 2;
 
-  for (int u = blockIdx.x; u < p.n_units && !aborted; u += G_stride) {
-    const int32_t* rec = p.plan + kPlanHeader + u * kPlanRecord;
-    const int b = rec[PR_B], h = rec[PR_H], tok0 = rec[PR_TOK_START];
-    const int L = rec[PR_LEN], nch = rec[PR_CHUNKS], coff = rec[PR_CHUNK_OFFSET];
-    const size_t sbase_g = ((size_t)b * p.Nv + h) * kD * kD;
+  for (int ii = blockIdx.x; ii < p.n_items && !aborted; ii += G_stride) {
+    const Item it = item_of(p, ii);
+    const int b = it.b, h = it.h, tok0 = it.tok0, L = it.L, coff = it.coff;
     const float a_h = expf(p.A_log[h]);
     const float lbl2 = p.lower_bound * kLog2e;
     float dtb[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) dtb[e] = p.dt_bias[h * kD + j0 + e];
 
-    // ---- state from initial_state: fp32 -> TMEM S, bf16 hi/lo -> TMEM state operand ----
+    // ---- start state (the item's: initial_state, a state slot, zeros or the identity):
+    //      fp32 -> TMEM S, bf16 hi/lo -> TMEM state operand ----
     {
       const int i = wq + lane;
 #pragma unroll 1
@@ -321,7 +408,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 16; c += 4) {
           float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (p.S0) x = __ldg(reinterpret_cast<const float4*>(p.S0 + sbase_g + (size_t)i * kD + col0 + c));
+          if (it.ident) {
+            const int d = i - (col0 + c);
+            x = make_float4(d == 0 ? 1.f : 0.f, d == 1 ? 1.f : 0.f, d == 2 ? 1.f : 0.f,
+                            d == 3 ? 1.f : 0.f);
+          } else if (it.s_in) {
+            x = *reinterpret_cast<const float4*>(it.s_in + (size_t)i * kD + col0 + c);
+          }
           fv[c] = __float_as_uint(x.x);
           fv[c + 1] = __float_as_uint(x.y);
           fv[c + 2] = __float_as_uint(x.z);
@@ -344,15 +437,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // beta logits of the next chunk (row tid), loaded one chunk ahead under the phase-5 MMAs
     __nv_bfloat16 bl_next = __float2bfloat16_rn(0.f);
-    if (tid < kChunk && tid < L) bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, tid)];
+    {
+      const int t = it.c_begin * kChunk + tid;
+      if (tid < kChunk && t < L) bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t)];
+    }
 
-    for (int c = 0; c < nch; ++c, ++gidx) {
+    for (int c = it.c_begin; c < it.c_end; ++c, ++gidx) {
       const int slot = gidx & 1;
       uint8_t* sq = sm + slot * SLOT_BYTES;  // slot base: q, g, v atoms at QGV_ATOM, k at K_ATOM
       const uint32_t as = sbase + slot * SLOT_BYTES;
       const int t0 = c * kChunk;
       const int n = min(kChunk, L - t0);
-      const bool last = (c == nch - 1);
+      const bool last = (c == it.c_end - 1);
       const bool tprof_on = p.tprof && blockIdx.x == 0 && tid == 0 && gidx < 64;
       KDA_TS(0);
 
@@ -510,7 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (Jb + 3 <= 3)
             *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 3) + r, j0)) =
                 pack4(b3[0], b3[1], b3[2], b3[3]);
-          if (!valid) *reinterpret_cast<uint2*>(sq + OFF_V + atom_off(QGV_ATOM, r, j0)) = make_uint2(0, 0);
+          if (!valid || it.zero_v)  // an M run treats v as zero
+            *reinterpret_cast<uint2*>(sq + OFF_V + atom_off(QGV_ATOM, r, j0)) = make_uint2(0, 0);
         }
       }
       fence_proxy_async_smem();
@@ -891,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint32_t*>(sq + OFF_V + off) = lo;
         }
       }
-      if (dbg) {  // per-chunk intermediates in the two-kernel workspace layout (fp32)
+      if (dbg && !it.zero_v) {  // per-chunk intermediates in the two-kernel workspace layout (fp32)
         float* dc = dbg + (size_t)(coff + c) * (kWsChunkBytes / 4);
         const int i = wq + lane;
         if (wg == 0) {
@@ -941,7 +1038,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bar_mma);
       }
-      if (c + 1 < nch && tid < kChunk && t0 + kChunk + tid < L)
+      if (c + 1 < it.c_end && tid < kChunk && t0 + kChunk + tid < L)
         bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t0 + kChunk + tid)];
       wait_mma();
       KDA_TS(7);
@@ -1000,7 +1097,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t vo[16];
         tmem_ld16(tl + TC_O + 16 * wg, vo);
         tmem_wait_ld();
-        if (n == kChunk) {
+        if (!it.write_out) {
+          // a segment-summary run: only its final state is kept
+        } else if (n == kChunk) {
           // full chunk: out tile [t][i] (128B-swizzled, as the out tensor map expects) in the free
           // Aop region, stored by TMA after the phase-8 barrier
           // (lanes i and i ^ 1 swap one value per token pair and write two adjacent columns)
@@ -1040,8 +1139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(tl + TC_SHI + col / 2, hi);
         tmem_st16(tl + TC_SLO + col / 2, lo);
-        if (last) {
-          float* dst = p.Sf + sbase_g + (size_t)i * kD + col;
+        if (last && it.s_out) {
+          float* dst = it.s_out + (size_t)i * kD + col;
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
             *reinterpret_cast<float4*>(dst + e) = make_float4(
@@ -1058,9 +1157,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncthreads();
       KDA_TS(10);
-      if (st_thread && n == kChunk) {
+      if (st_thread && n == kChunk && it.write_out) {
         int qc1, qc2, oc1, oc2;
-        const UnitRec ur{b, h, 0, tok0, nch};
+        const LoadRec ur{b, h, 0, tok0, 0, 0};
         chunk_coords(p, ur, c, qc1, qc2, oc1, oc2);
         const int half = warp - 9;
         tma_store_3d(&maps.o, sbase + SM_OSTG + half * 8192, 64 * half, oc1, oc2);
@@ -1072,7 +1171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // rows past the valid length (BNSD/BSND storage padding) are defined as zero
-    if (!aborted && p.layout != KDA_LAYOUT_TND) {
+    if (!aborted && it.pad && p.layout != KDA_LAYOUT_TND) {
       for (int e = tid; e < (p.S - L) * 16; e += kThreads) {
         const int t = L + (e >> 4), q8 = (e & 15) * 8;
         *reinterpret_cast<uint4*>(p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t) + q8) =
@@ -1138,7 +1237,8 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
       !make_map(&m.g, p.g, p.layout, p.B, p.Nv, p.S) ||
       !make_map(&m.o, p.out, p.layout, p.B, p.Nv, p.S))
     return cudaErrorInvalidValue;
-  const int grid = p.n_units < num_sms ? p.n_units : num_sms;
+  if (p.n_items < 1) return cudaSuccess;
+  const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   kda_fused_kernel<<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
   return cudaGetLastError();
 }

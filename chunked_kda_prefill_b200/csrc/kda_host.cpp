@@ -38,6 +38,23 @@ kda_status_t validate_shape(const kda_shape_t* s) {
   return KDA_OK;
 }
 
+SegCounts seg_counts(const int32_t* p) {
+  SegCounts c{0, 0, 0};
+  const int32_t seg = p[PH_SEG_CHUNKS];
+  if (seg <= 0) return c;
+  for (int u = 0; u < p[PH_UNITS]; ++u) {
+    const int32_t nseg = unit_segments(p[kPlanHeader + u * kPlanRecord + PR_CHUNKS], seg);
+    c.items_a += 2LL * nseg - 1;  // the first segment from the true state; R and M runs after
+    c.items_c += nseg - 1;        // outputs of every segment after the first
+  }
+  c.slots = c.items_c;
+  return c;
+}
+
+size_t fused_workspace_bytes(const int32_t* p) {
+  return kWsHeaderBytes + (size_t)seg_counts(p).slots * kSlotBytes;
+}
+
 kda_status_t validate_plan(const int32_t* p, size_t n, const kda_shape_t* s) {
   if (!p) return KDA_ERR_NULL;
   if (n < (size_t)kPlanHeader) return KDA_ERR_PLAN;
@@ -47,6 +64,7 @@ kda_status_t validate_plan(const int32_t* p, size_t n, const kda_shape_t* s) {
   const long long need = kPlanHeader + (long long)p[PH_UNITS] * kPlanRecord;
   if (p[PH_UNITS] < 1 || (long long)n < need) return KDA_ERR_PLAN;
   if (plan_checksum(p, (size_t)need) != p[PH_CHECKSUM]) return KDA_ERR_PLAN;
+  if (p[PH_SEG_CHUNKS] < 0) return KDA_ERR_PLAN;
   if (s) {
     if (p[PH_LAYOUT] != s->layout || p[PH_B] != s->B || p[PH_NQK] != s->Nqk ||
         p[PH_NV] != s->Nv || p[PH_S] != s->S || p[PH_D] != s->D ||
@@ -93,8 +111,21 @@ extern "C" kda_status_t kda_plan_size(const kda_shape_t* shape, size_t* n_int32)
   return KDA_OK;
 }
 
-extern "C" kda_status_t kda_plan(const kda_shape_t* shape, const int32_t* cu, int32_t num_sms,
-                                 int32_t* plan, size_t n_int32) {
+namespace {
+
+// The segment length the default schedule picks: units run whole unless they would leave more
+// than half the SMs idle and are long enough to split; then segments are sized so that the
+// first pass (about two work items per segment) fills the SMs once.  At least 2 chunks per
+// segment: shorter segments cost more in the extra passes than they save.
+int32_t auto_segment_chunks(long long units, long long total_chunks, int32_t max_chunks,
+                            int32_t num_sms) {
+  if (units * 2 > num_sms || max_chunks < 8) return 0;
+  const long long half = std::max(1, num_sms / 2);
+  return (int32_t)std::max(2LL, (total_chunks + half - 1) / half);
+}
+
+kda_status_t plan_impl(const kda_shape_t* shape, const int32_t* cu, int32_t num_sms,
+                       int32_t seg_request, int32_t* plan, size_t n_int32) {
   kda_status_t st = validate_shape(shape);
   if (st != KDA_OK) return st;
   if (!plan) return KDA_ERR_NULL;
@@ -154,6 +185,18 @@ extern "C" kda_status_t kda_plan(const kda_shape_t* shape, const int32_t* cu, in
     maxc = std::max(maxc, units[i].chunks);
   }
   if (total > INT_MAX) return KDA_ERR_SHAPE;
+  // segment length: explicit request (> 0), none (0), or the default policy (< 0)
+  const int32_t seg = seg_request >= 0 ? seg_request
+                                       : auto_segment_chunks((long long)units.size(), total, maxc,
+                                                             num_sms);
+  long long seg_base = 0;
+  for (size_t i = 0; i < units.size(); ++i) {
+    int32_t* r = plan + kPlanHeader + i * kPlanRecord;
+    r[PR_SEG_BASE] = (int32_t)seg_base;
+    if (seg > 0) seg_base += unit_segments(units[i].chunks, seg) - 1;
+    if (seg_base > INT_MAX / 4) return KDA_ERR_SHAPE;
+  }
+  plan[PH_SEG_CHUNKS] = seg;
   plan[PH_MAGIC] = kPlanMagic;
   plan[PH_VERSION] = kPlanVersion;
   plan[PH_HEADER_WORDS] = kPlanHeader;
@@ -172,10 +215,25 @@ extern "C" kda_status_t kda_plan(const kda_shape_t* shape, const int32_t* cu, in
   return KDA_OK;
 }
 
+}  // namespace
+
+extern "C" kda_status_t kda_plan(const kda_shape_t* shape, const int32_t* cu, int32_t num_sms,
+                                 int32_t* plan, size_t n_int32) {
+  return plan_impl(shape, cu, num_sms, -1, plan, n_int32);
+}
+
+extern "C" kda_status_t kda_plan_segmented(const kda_shape_t* shape, const int32_t* cu,
+                                           int32_t num_sms, int32_t segment_chunks,
+                                           int32_t* plan, size_t n_int32) {
+  if (segment_chunks < 0) return KDA_ERR_SHAPE;
+  return plan_impl(shape, cu, num_sms, segment_chunks, plan, n_int32);
+}
+
 extern "C" kda_status_t kda_workspace_size(const int32_t* plan, size_t n, size_t* bytes) {
   if (!bytes) return KDA_ERR_NULL;
   kda_status_t st = validate_plan(plan, n, nullptr);
   if (st != KDA_OK) return st;
-  *bytes = kWsHeaderBytes;  // the fused kernel keeps only its status word in the workspace
+  // the status word, plus the state slots of a segmented schedule
+  *bytes = fused_workspace_bytes(plan);
   return KDA_OK;
 }

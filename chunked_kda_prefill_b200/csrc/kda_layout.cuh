@@ -28,6 +28,10 @@ struct Params {
   __nv_bfloat16* out;
   float* Sf;
   unsigned long long* tprof;  // optional: CTA 0 records clock64() at phase boundaries
+  // work items of this launch: mode 0 = whole units; under a segmented plan (seg_chunks > 0)
+  // mode 1 = the segment-summary pass, mode 2 = the output pass (see kda_plan_segmented)
+  int mode, seg_chunks, n_items;
+  float* states;  // the segmented schedule's state slots (workspace after its header)
 };
 
 // Element offset of the D-vector of (sequence b, head hx of NX heads, token t of the sequence).
@@ -63,6 +67,9 @@ cudaError_t launch_simt(const Params& p, int total_chunks, cudaStream_t stream);
 // The fused tcgen05 path (kda_fused.cu): needs kWsHeaderBytes of workspace.  A non-null `dbg`
 // receives every chunk's intermediates in the two-kernel workspace layout (test aid).
 cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream);
+// The segmented schedule's middle kernel: every unit's segment start states from the segment
+// summaries (S_{s+1} = S_s M_s + R_s, fp32).
+cudaError_t launch_combine(const Params& p, cudaStream_t stream);
 
 enum ForwardPath : int { PATH_FUSED = 0, PATH_SIMT = 1 };
 

@@ -100,11 +100,31 @@ KDA_API kda_status_t kda_plan_size(const kda_shape_t* shape, size_t* n_int32);
  *     sequence b then occupies storage rows [0, len_b) of slot b (FlashKDA README 约束说明).
  *   num_sms: multiprocessor count of the target device (>= 1); recorded in the plan.
  *   plan, n_int32: host output buffer and its capacity in int32 words.
- * Units are ordered longest first.  Pure host code; never touches the GPU. */
+ * Units are ordered longest first.  Pure host code; never touches the GPU.
+ *
+ * Schedule: when the units would leave more than half of num_sms idle and the longest has at
+ * least 8 chunks, the plan is segmented (see kda_plan_segmented) with segments sized so that
+ * about num_sms work items run at once; otherwise every unit runs whole on one CTA. */
 KDA_API kda_status_t kda_plan(const kda_shape_t* shape, const int32_t* cu_seqlens_host, int32_t num_sms,
                       int32_t* plan, size_t n_int32);
 
-/* Device workspace bytes kda_forward needs for this plan (host plan).  Always >= 256. */
+/* kda_plan with an explicit schedule: segment_chunks == 0 runs every unit whole;
+ * segment_chunks > 0 cuts every unit into segments of that many 64-token chunks (the last one
+ * shorter) that run in parallel, the chunk-parallel form of the state scan.  Per chunk the
+ * state update is affine, S_next = S M + R with M = Diag(gamma_C) - W^T K^ and R = U^T K^
+ * (the FlashKDA README's chunk equations, 功能说明, rearranged), so a segment maps its start
+ * state S to S M_seg + R_seg.  kda_forward then runs three kernels: (1) every segment's
+ * (M_seg, R_seg) as the final state from S = I with v = 0 and from S = 0 (the first segment of
+ * a unit runs from its true initial state instead, writing its outputs); (2) the segment start
+ * states, S_{s+1} = S_s M_s + R_s in fp32; (3) every later segment again from its start state,
+ * writing outputs and, for a unit's last segment, final_state.  Results agree with the whole-unit
+ * schedule within rounding.  segment_chunks < 0 is KDA_ERR_SHAPE. */
+KDA_API kda_status_t kda_plan_segmented(const kda_shape_t* shape, const int32_t* cu_seqlens_host,
+                                        int32_t num_sms, int32_t segment_chunks, int32_t* plan,
+                                        size_t n_int32);
+
+/* Device workspace bytes kda_forward needs for this plan (host plan): 256, plus 192 KiB per
+ * segment after each unit's first under a segmented schedule. */
 KDA_API kda_status_t kda_workspace_size(const int32_t* plan_host, size_t n_int32, size_t* bytes);
 
 /* The forward pass (FlashKDA README, flash_kda): writes out and final_state.

@@ -180,3 +180,63 @@ def test_decode_argument_checks(L):
     # checks need a GPU (none here -> CUDA/device error)
     assert _dec(L, s1=0x20000000) in (11, 13)
     assert _dec(L, s0=None) in (11, 13)
+
+
+def _plan_seg(L, shape, seg, cu=None, sms=148):
+    n = ctypes.c_size_t(0)
+    assert L.kda_plan_size(ctypes.byref(shape), ctypes.byref(n)) == 0
+    buf = np.zeros(n.value, dtype=np.int32)
+    cu_p = None
+    if cu is not None:
+        cu = np.asarray(cu, dtype=np.int32)
+        cu_p = cu.ctypes.data_as(P_I32)
+    st = L.kda_plan_segmented(ctypes.byref(shape), cu_p, sms, seg, buf.ctypes.data_as(P_I32),
+                              buf.size)
+    return st, buf
+
+
+def _ws(L, p):
+    ws = ctypes.c_size_t(0)
+    assert L.kda_workspace_size(p.ctypes.data_as(P_I32), p.size, ctypes.byref(ws)) == 0
+    return ws.value
+
+
+def test_default_schedule_segments_only_few_long_units(L):
+    # 3 units of 128 chunks on 148 SMs: segmented, ~2 work items per segment fill the SMs once
+    st, p = _plan(L, _shape(layout=0, B=1, Nqk=3, Nv=3, S=8192))
+    assert st == 0 and p[14] == 6
+    # 128 units of 256 chunks: whole units
+    st, p = _plan(L, _shape(layout=0, B=4, Nqk=32, Nv=32, S=16384))
+    assert st == 0 and p[14] == 0 and _ws(L, p) == 256
+    # one unit of 4 chunks: too short to split
+    st, p = _plan(L, _shape(layout=0, B=1, Nqk=1, Nv=1, S=256))
+    assert st == 0 and p[14] == 0
+    # few SMs: 3 units already fill them
+    st, p = _plan(L, _shape(layout=0, B=1, Nqk=3, Nv=3, S=8192), sms=4)
+    assert st == 0 and p[14] == 0
+
+
+def test_segmented_plan_state_slots(L):
+    # varlen BSND: lengths 4000 and 2777 -> 63 and 44 chunks per unit, 16 heads each
+    sh = _shape(layout=1, B=2, Nqk=4, Nv=16, S=4000)
+    st, p = _plan_seg(L, sh, 8, cu=[0, 4000, 6777])
+    assert st == 0 and p[14] == 8
+    recs = p[16:].reshape(32, 8)
+    nseg = [(int(r[5]) + 7) // 8 for r in recs]
+    assert sorted(set(nseg)) == [6, 8]
+    # PR_SEG_BASE: prefix sum of (segments - 1) over the earlier units, in plan order
+    expect, acc = [], 0
+    for s in nseg:
+        expect.append(acc)
+        acc += s - 1
+    assert [int(r[7]) for r in recs] == expect
+    assert _ws(L, p) == 256 + acc * 3 * 128 * 128 * 4
+    # segment_chunks = 0 is the whole-unit schedule; negative is rejected
+    st, p0 = _plan_seg(L, sh, 0, cu=[0, 4000, 6777])
+    assert st == 0 and p0[14] == 0 and _ws(L, p0) == 256
+    assert _plan_seg(L, sh, -1, cu=[0, 4000, 6777])[0] == 3
+    # a corrupted segment length fails validation
+    bad = p.copy()
+    bad[14] = -2
+    ws = ctypes.c_size_t(0)
+    assert L.kda_workspace_size(bad.ctypes.data_as(P_I32), bad.size, ctypes.byref(ws)) == 8
