@@ -261,7 +261,8 @@ def run_ours(args, rank, world):
         host[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).pin_memory()
     d = {n: t.to(dev) for n, t in host.items()}
     cu = w.cu_seqlens if (w.layout == "TND" or any(L != w.S for L in w.lengths)) else None
-    plan = kda.plan(d["q"], d["v"], d["initial_state"], w.layout, cu_seqlens=cu)
+    plan = kda.plan(d["q"], d["v"], d["initial_state"], w.layout, cu_seqlens=cu,
+                    segment_chunks=None if args.segment_chunks < 0 else args.segment_chunks)
     ws = plan.workspace()
     out = torch.empty_like(d["v"])
     fs = torch.empty((w.B, w.Nv, w.D, w.D), dtype=torch.float32, device=dev)
@@ -347,7 +348,10 @@ def run_ours(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 inputs, random-init A_log/dt_bias)",
-            "config": _config(w, world), "clocks": clk.report(), "e2e": e2e,
+            "config": dict(_config(w, world), schedule=(
+                f"segments of {plan.segment_chunks} chunks (chunk-parallel scan)"
+                if plan.segment_chunks > 0 else "whole units, one CTA each")),
+            "clocks": clk.report(), "e2e": e2e,
             "gpu_launches": args.steps * kda.kernels_per_forward(plan),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": ncu_traffic(w.name),
@@ -399,6 +403,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)
+    ap.add_argument("--segment-chunks", type=int, default=-1,
+                    help="schedule: -1 the planner's choice, 0 whole units, n > 0 segments of n "
+                         "chunks (chunk-parallel scan)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = _env_int("RANK", 0)
