@@ -7,8 +7,9 @@
 // R_s of every segment s >= 1 in its state slot, and the true start state of segment 1 (the end
 // state of segment 0).  Here, per unit and in segment order,
 //     S_{s+1} = S_s M_s + R_s        (fp32, 128 x 128 x 128 per step)
-// for s = 1 .. nseg-2.  Rows of S are independent, so a unit's 128 rows are split over 8 CTAs
-// of 16 rows; each CTA streams M_s through shared memory in 16-row slices.
+// for s = 1 .. nseg-2.  Rows of S are independent, so a unit's 128 rows are split over 16 CTAs
+// of 8 rows.  Every M_s is known before the kernel starts, so M_{s+1} streams into shared memory
+// (cp.async, double-buffered) while step s computes; only S_s is carried from step to step.
 #include <cuda_runtime.h>
 
 #include "kda_internal.h"
@@ -17,78 +18,99 @@
 namespace kda {
 namespace {
 
-constexpr int kRows = 16;      // state rows per CTA
-constexpr int kKSlice = 16;    // rows of M per shared-memory slice
-constexpr int kThreadsC = 256;  // thread = (row, 8-column group)
+constexpr int kRowsC = 8;        // state rows per CTA
+constexpr int kThreadsC = 256;   // thread = (4-row group, column)
+constexpr size_t kCombineSmem = (2 * kD * kD + kRowsC * kD) * sizeof(float);
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_one() {  // all but the newest group complete
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 __global__ void __launch_bounds__(kThreadsC) kda_combine_kernel(const Params p) {
-  __shared__ __align__(16) float sS[kRows][kD];
-  __shared__ __align__(16) float sM[kKSlice][kD];
-  const int u = blockIdx.x, r0 = blockIdx.y * kRows;
+  extern __shared__ __align__(16) float csm[];
+  float* sM = csm;                 // [2][128][128]: M of the current and the next step
+  float* sS = csm + 2 * kD * kD;   // [8][128]: this CTA's rows of S_s
+  const int u = blockIdx.x, r0 = blockIdx.y * kRowsC;
   const int32_t* rec = p.plan + kPlanHeader + u * kPlanRecord;
   const int seg = p.seg_chunks;
   const int nseg = (rec[PR_CHUNKS] + seg - 1) / seg;
   const int base = rec[PR_SEG_BASE];
   if (nseg < 3) return;  // S_1 comes from the first pass; nothing to chain
-  const int tid = threadIdx.x, r = tid >> 4, c0 = (tid & 15) * 8;
+  const int tid = threadIdx.x, rg = tid >> 7, col = tid & (kD - 1);
   auto slot = [&](int sl, int part) {
     return p.states + (size_t)sl * kSlotFloats + (size_t)part * kD * kD;
   };
-  // S_1 rows
-  for (int e = tid; e < kRows * kD / 4; e += kThreadsC) {
-    const int rr = e / (kD / 4), cc = (e % (kD / 4)) * 4;
-    *reinterpret_cast<float4*>(&sS[rr][cc]) =
-        *reinterpret_cast<const float4*>(slot(base, SLOT_START) + (size_t)(r0 + rr) * kD + cc);
-  }
-  __syncthreads();
-  for (int s = 1; s <= nseg - 2; ++s) {
-    const float* M = slot(base + s - 1, SLOT_M);
-    const float* R = slot(base + s - 1, SLOT_R) + (size_t)(r0 + r) * kD + c0;
-    float acc[8];
-    {
-      const float4 a = *reinterpret_cast<const float4*>(R);
-      const float4 b = *reinterpret_cast<const float4*>(R + 4);
-      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
-      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
-    }
-    for (int k0 = 0; k0 < kD; k0 += kKSlice) {
-      for (int e = tid; e < kKSlice * kD / 4; e += kThreadsC) {
-        const int kk = e / (kD / 4), cc = (e % (kD / 4)) * 4;
-        *reinterpret_cast<float4*>(&sM[kk][cc]) =
-            *reinterpret_cast<const float4*>(M + (size_t)(k0 + kk) * kD + cc);
-      }
-      __syncthreads();
+  auto load_m = [&](int s) {  // M_s -> buffer (s - 1) & 1, 16 x 16 bytes per thread
+    const float* src = slot(base + s - 1, SLOT_M);
+    float* dst = sM + (size_t)((s - 1) & 1) * kD * kD;
+    for (int e = tid; e < kD * kD / 4; e += kThreadsC) cp_async16(dst + 4 * e, src + 4 * e);
+  };
+  auto load_r = [&](int s, float (&r)[4]) {  // this thread's 4 entries of R_s
+    const float* src = slot(base + s - 1, SLOT_R);
 #pragma unroll
-      for (int kk = 0; kk < kKSlice; ++kk) {
-        const float sv = sS[r][k0 + kk];
-        const float4 a = *reinterpret_cast<const float4*>(&sM[kk][c0]);
-        const float4 b = *reinterpret_cast<const float4*>(&sM[kk][c0 + 4]);
-        acc[0] = fmaf(sv, a.x, acc[0]);
-        acc[1] = fmaf(sv, a.y, acc[1]);
-        acc[2] = fmaf(sv, a.z, acc[2]);
-        acc[3] = fmaf(sv, a.w, acc[3]);
-        acc[4] = fmaf(sv, b.x, acc[4]);
-        acc[5] = fmaf(sv, b.y, acc[5]);
-        acc[6] = fmaf(sv, b.z, acc[6]);
-        acc[7] = fmaf(sv, b.w, acc[7]);
+    for (int i = 0; i < 4; ++i) r[i] = src[(size_t)(r0 + 4 * rg + i) * kD + col];
+  };
+
+  for (int e = tid; e < kRowsC * kD / 4; e += kThreadsC)
+    *reinterpret_cast<float4*>(sS + 4 * e) =
+        *reinterpret_cast<const float4*>(slot(base, SLOT_START) + (size_t)r0 * kD + 4 * e);
+  load_m(1);
+  cp_async_commit();
+  float r_cur[4];
+  load_r(1, r_cur);
+
+  for (int s = 1; s <= nseg - 2; ++s) {
+    if (s + 1 <= nseg - 2) load_m(s + 1);
+    cp_async_commit();  // (an empty group on the last step keeps the wait count uniform)
+    float r_next[4] = {0.f, 0.f, 0.f, 0.f};
+    if (s + 1 <= nseg - 2) load_r(s + 1, r_next);
+    cp_async_wait_one();
+    __syncthreads();  // M_s (everyone's copies) and S_s are in shared memory
+    const float* M = sM + (size_t)((s - 1) & 1) * kD * kD;
+    float acc[4] = {r_cur[0], r_cur[1], r_cur[2], r_cur[3]};
+#pragma unroll 4
+    for (int k = 0; k < kD; k += 4) {
+      const float m0 = M[(k + 0) * kD + col], m1 = M[(k + 1) * kD + col];
+      const float m2 = M[(k + 2) * kD + col], m3 = M[(k + 3) * kD + col];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 sv = *reinterpret_cast<const float4*>(sS + (4 * rg + i) * kD + k);
+        acc[i] = fmaf(sv.x, m0, fmaf(sv.y, m1, fmaf(sv.z, m2, fmaf(sv.w, m3, acc[i]))));
       }
-      __syncthreads();
     }
-    // S_{s+1}: to its slot, and to shared memory for the next step
-    float* dst = slot(base + s, SLOT_START) + (size_t)(r0 + r) * kD + c0;
-    *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    *reinterpret_cast<float4*>(&sS[r][c0]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    *reinterpret_cast<float4*>(&sS[r][c0 + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    __syncthreads();
+    __syncthreads();  // every read of S_s and of this M buffer is done
+    float* dst = slot(base + s, SLOT_START);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      dst[(size_t)(r0 + 4 * rg + i) * kD + col] = acc[i];
+      sS[(4 * rg + i) * kD + col] = acc[i];
+      r_cur[i] = r_next[i];
+    }
   }
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const Params& p, cudaStream_t stream) {
-  const dim3 grid((unsigned)p.n_units, kD / kRows);
-  kda_combine_kernel<<<grid, kThreadsC, 0, stream>>>(p);
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(kda_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kCombineSmem);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  const dim3 grid((unsigned)p.n_units, kD / kRowsC);
+  kda_combine_kernel<<<grid, kThreadsC, kCombineSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
