@@ -824,11 +824,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const int kq = lane & 3, tile = warp * 8 + (lane >> 2);
         const int ra = 32 + 4 * (tile >> 4), cb = 2 * (tile & 15);
+        // X_(0:32, 0:32) is zero in rows 0-15 of columns 16-31, so tiles right of column 16 (odd
+        // warps) need only m = 1 here; X_(32:64, 32:64) is zero in columns 48-63 of rows 32-47,
+        // so rows below 48 (warps 0-7) need only m = 0 in the second product.
+        const int m_lo = (warp & 1) ? 1 : 0, m_hi = (warp < 8) ? 1 : 2;
         float acc[4][2];
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
+#pragma unroll 1
+        for (int m = m_lo; m < 2; ++m) {
           const int kb = 4 * kq + 16 * m;
           float tv[4][4];
 #pragma unroll
@@ -861,8 +865,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
+#pragma unroll 1
+        for (int m = 0; m < m_hi; ++m) {
           const int kb = 4 * kq + 16 * m;
           float xv4[4][4];
 #pragma unroll
