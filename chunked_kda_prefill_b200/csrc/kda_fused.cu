@@ -71,13 +71,15 @@ constexpr uint32_t QGV_ATOM = 24576;  // distance between the two column halves 
 constexpr uint32_t K_ATOM = 8192;
 constexpr uint32_t SM_AOP = 131072;   // [128 rows][128] bf16, 2 atoms of 16 KB; after phase 2:
 constexpr uint32_t SM_XSOL = SM_AOP;  //   [Xsol hi ; Xsol lo] 128 rows x 64 cols (16 KB)
-constexpr uint32_t SM_OSTG = SM_AOP;  //   phase 8: out tile [64 tokens][128] for the TMA store
+constexpr uint32_t SM_GT = SM_AOP;    //   from phase 5: the next chunk's in-warp gate cumsums,
+                                      //   fp32 [64][128] (read back in its phase 1)
 constexpr uint32_t SM_BT = 163840;    // [B^(0); B^(1); B^(2); B^(3)]: one 160-row tile; the solve
-constexpr uint32_t BT_ROWS = 160;     //   scratch in phase 3
-constexpr uint32_t SM_KLO = 204800;   // K^ lo part [64][128] (phases 2-7); phase 1: constants
-constexpr uint32_t SM_CST = SM_KLO;   //   fp32 [7][4 blocks][128]
-constexpr uint32_t SM_AQK = 221184;   // [64][64] bf16 (phases 3-7); phase 1: warp totals
-constexpr uint32_t SM_WTOT = SM_AQK;  //   fp32 [16 warps][128]
+constexpr uint32_t BT_ROWS = 160;     //   scratch in phase 3; from phase 5 the next chunk's
+constexpr uint32_t SM_WTOT = SM_BT;   //   warp totals / prefixes fp32 [16][128] and
+constexpr uint32_t SM_CST = SM_BT + 8192;  // reference constants fp32 [7][4 blocks][128]
+constexpr uint32_t SM_KLO = 204800;   // K^ lo part [64][128] (phases 2-7); phase 8 until the
+constexpr uint32_t SM_OSTG = SM_KLO;  //   next chunk's phase 2: the out tile for the TMA store
+constexpr uint32_t SM_AQK = 221184;   // [64][64] bf16 (phases 3-7)
 constexpr uint32_t SM_GC = 229376;    // fp32 [128]: 2^G_last
 constexpr uint32_t SM_BETA = 229888;  // fp32 [64]
 constexpr uint32_t SM_BAR = 230144;   // raw_full[2], mma
@@ -303,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_FLAG);
   float* wtot = reinterpret_cast<float*>(sm + SM_WTOT);
   float* cst = reinterpret_cast<float*>(sm + SM_CST);
+  float* gtile = reinterpret_cast<float*>(sm + SM_GT);
   float* gcs = reinterpret_cast<float*>(sm + SM_GC);
   float* beta_s = reinterpret_cast<float*>(sm + SM_BETA);
 
@@ -435,11 +438,82 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
 
-    // beta logits of the next chunk (row tid), loaded one chunk ahead under the phase-5 MMAs
+    // The front of phase 1 of chunk cc (ring slot of the gi-th chunk of this CTA): wait for its
+    // tiles; gate activation and the in-thread cumsum of this thread's 4 rows -> the G tile,
+    // warp totals -> wtot; beta.  For every chunk after an item's first it runs under the
+    // previous chunk's phase-5 MMAs (the G tile and wtot regions are free from then on).
+    auto front_gate = [&](int cc, uint32_t gi, __nv_bfloat16 blog) {
+      const int nn = min(kChunk, L - cc * kChunk);
+      const uint8_t* sg_tile = sm + (gi & 1) * SLOT_BYTES + OFF_G;
+      if (!mbar_wait_bounded(sbase + SM_BAR + 8u * (gi & 1), (gi >> 1) & 1u, kWaitLimit)) fail();
+      // g_act * log2(e) = lb log2(e) / (1 + 2^(-log2(e) e^A_log (g_raw + dt_bias)))
+      const float ca = -a_h * kLog2e;
+      float G[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = r0 + i;
+        float gv[4];
+        unpack4(*reinterpret_cast<const uint2*>(sg_tile + atom_off(QGV_ATOM, r, j0)), gv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float sgm = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
+          G[i][e] = (r < nn) ? sgm : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (i > 0)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) G[i][e] += G[i - 1][e];
+        *reinterpret_cast<float4*>(gtile + (r0 + i) * kD + j0) =
+            make_float4(G[i][0], G[i][1], G[i][2], G[i][3]);
+      }
+      *reinterpret_cast<float4*>(wtot + warp * kD + j0) =
+          make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+      if (tid < kChunk)
+        beta_s[tid] = (tid < nn) ? __fdividef(1.0f, 1.0f + __expf(-__bfloat162float(blog))) : 0.0f;
+    };
+    // Column tid (< 128): exclusive prefix of the 16 warp totals (in place); the block reference
+    // rows (G at rows 15, 31, 47, 63) and from them the per-block constants of the
+    // factorisation; 2^G_last.  Runs under the previous chunk's phase-7 MMAs (after the first).
+    auto front_scan = [&]() {
+      if (tid >= kD) return;
+      const int j = tid;
+      float run = 0.f, ref[4];
+#pragma unroll
+      for (int w2 = 0; w2 < 16; ++w2) {
+        const float t = wtot[w2 * kD + j];
+        wtot[w2 * kD + j] = run;
+        run += t;
+        if ((w2 & 3) == 3) ref[w2 >> 2] = run;
+      }
+#pragma unroll
+      for (int I = 0; I < 4; ++I) {
+        const float refI = (I == 0) ? 0.f : ref[I - 1];
+        const float ge = ref[I];
+        cst[(CST_REF * 4 + I) * kD + j] = refI;
+        cst[(CST_GE * 4 + I) * kD + j] = ge;
+        cst[(CST_P2REF * 4 + I) * kD + j] = ex2(refI);
+        cst[(CST_KFAC * 4 + I) * kD + j] = ex2(ref[3] - ge);
+        cst[(CST_CDIAG * 4 + I) * kD + j] = ex2(refI - ge);
+        cst[(CST_C2 * 4 + I) * kD + j] = (I <= 1) ? ex2(ref[I + 1] - ge) : 0.f;
+        cst[(CST_C3 * 4 + I) * kD + j] = (I == 0) ? ex2(ref[2] - ge) : 0.f;
+      }
+      gcs[j] = ex2(ref[3]);
+    };
+
+    // beta logits (row tid): the item's first chunk now, each later chunk one chunk ahead
     __nv_bfloat16 bl_next = __float2bfloat16_rn(0.f);
     {
       const int t = it.c_begin * kChunk + tid;
-      if (tid < kChunk && t < L) bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t)];
+      __nv_bfloat16 bl_first = __float2bfloat16_rn(0.f);
+      if (tid < kChunk && t < L) bl_first = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t)];
+      if (tid < kChunk && t + kChunk < L)
+        bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t + kChunk)];
+      front_gate(it.c_begin, gidx, bl_first);
+      __syncthreads();
+      front_scan();
+      __syncthreads();
     }
 
     for (int c = it.c_begin; c < it.c_end; ++c, ++gidx) {
@@ -452,69 +526,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool tprof_on = p.tprof && blockIdx.x == 0 && tid == 0 && gidx < 64;
       KDA_TS(0);
 
-      // =================== phase 1: prologue and operand tiles ===================
-      const __nv_bfloat16 blog = bl_next;
-      if (!mbar_wait_bounded(sbase + SM_BAR + 8u * slot, (gidx >> 1) & 1u, kWaitLimit)) fail();
-      KDA_TS(1);
-
+      // =================== phase 1: operand tiles ===================
       float G[4][4];
+      float k4[CST_N][4];
       {
-        // g_act * log2(e) = lb log2(e) / (1 + 2^(-log2(e) e^A_log (g_raw + dt_bias)))
-        const float ca = -a_h * kLog2e;
+        // this thread's rows of G (in-warp cumsum + the warp prefix) and its block's constants,
+        // all read before any thread overwrites the regions they live in
+        const float4 pre = *reinterpret_cast<const float4*>(wtot + warp * kD + j0);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int r = r0 + i;
-          float gv[4];
-          unpack4(*reinterpret_cast<const uint2*>(sq + OFF_G + atom_off(QGV_ATOM, r, j0)), gv);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float sg = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
-            G[i][e] = (r < n) ? sg : 0.0f;
-          }
+          const float4 x = *reinterpret_cast<const float4*>(gtile + (r0 + i) * kD + j0);
+          G[i][0] = x.x + pre.x;
+          G[i][1] = x.y + pre.y;
+          G[i][2] = x.z + pre.z;
+          G[i][3] = x.w + pre.w;
         }
-#pragma unroll
-        for (int i = 1; i < 4; ++i)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) G[i][e] += G[i - 1][e];
-        *reinterpret_cast<float4*>(wtot + warp * kD + j0) =
-            make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
-      }
-      if (tid < kChunk)
-        beta_s[tid] = (tid < n) ? __fdividef(1.0f, 1.0f + __expf(-__bfloat162float(blog))) : 0.0f;
-      __syncthreads();
-      KDA_TS(11);
-      if (tid < kD) {
-        // column tid: exclusive prefix of the 16 warp totals (in place); the block reference rows
-        // (G at rows 15, 31, 47, 63) and from them the per-block constants of the factorisation
-        const int j = tid;
-        float run = 0.f, ref[4];
-#pragma unroll
-        for (int w2 = 0; w2 < 16; ++w2) {
-          const float t = wtot[w2 * kD + j];
-          wtot[w2 * kD + j] = run;
-          run += t;
-          if ((w2 & 3) == 3) ref[w2 >> 2] = run;
-        }
-#pragma unroll
-        for (int I = 0; I < 4; ++I) {
-          const float refI = (I == 0) ? 0.f : ref[I - 1];
-          const float ge = ref[I];
-          cst[(CST_REF * 4 + I) * kD + j] = refI;
-          cst[(CST_GE * 4 + I) * kD + j] = ge;
-          cst[(CST_P2REF * 4 + I) * kD + j] = ex2(refI);
-          cst[(CST_KFAC * 4 + I) * kD + j] = ex2(ref[3] - ge);
-          cst[(CST_CDIAG * 4 + I) * kD + j] = ex2(refI - ge);
-          cst[(CST_C2 * 4 + I) * kD + j] = (I <= 1) ? ex2(ref[I + 1] - ge) : 0.f;
-          cst[(CST_C3 * 4 + I) * kD + j] = (I == 0) ? ex2(ref[2] - ge) : 0.f;
-        }
-        gcs[j] = ex2(ref[3]);
-      }
-      if (st_thread) tma_store_wait_read();  // the out tile staged in the Aop region was read
-      __syncthreads();
-      KDA_TS(12);
-      uint2 khlo[4];  // K^ lo parts of this thread's rows, stored once the intra MMA is done
-      {
-        float k4[CST_N][4];
 #pragma unroll
         for (int v = 0; v < CST_N; ++v) {
           const float4 x = *reinterpret_cast<const float4*>(cst + (v * 4 + Jb) * kD + j0);
@@ -523,14 +549,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           k4[v][2] = x.z;
           k4[v][3] = x.w;
         }
-        {
-          const float4 x = *reinterpret_cast<const float4*>(wtot + warp * kD + j0);
-          const float pre[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) G[i][e] += pre[e];
-        }
+      }
+      __syncthreads();
+      KDA_TS(12);
+      uint2 khlo[4];  // K^ lo parts of this thread's rows, stored once the intra MMA is done
+      {
         float rqv[4], rkv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -610,6 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint2*>(sq + OFF_V + atom_off(QGV_ATOM, r, j0)) = make_uint2(0, 0);
         }
       }
+      if (st_thread) tma_store_wait_read();  // the previous out tile (in the K^ lo region) was read
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
@@ -1042,8 +1066,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bar_mma);
       }
-      if (c + 1 < it.c_end && tid < kChunk && t0 + kChunk + tid < L)
-        bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t0 + kChunk + tid)];
+      if (c + 1 < it.c_end) {
+        // the next chunk's gate and cumsum under these MMAs, then its successor's beta load
+        front_gate(c + 1, gidx + 1, bl_next);
+        const int t2 = t0 + 2 * kChunk + tid;
+        if (c + 2 < it.c_end && tid < kChunk && t2 < L)
+          bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t2)];
+      }
       wait_mma();
       KDA_TS(7);
       tc_fence_after();
@@ -1090,6 +1119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_mma);
       }
       if (lane == 0 && warp >= 1 && warp <= 6) issue_planned(warp - 1);  // q/g/v of this slot are free
+      if (c + 1 < it.c_end) front_scan();  // the next chunk's column scan under these MMAs
       wait_mma();
       KDA_TS(9);
       tc_fence_after();
@@ -1105,7 +1135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // a segment-summary run: only its final state is kept
         } else if (n == kChunk) {
           // full chunk: out tile [t][i] (128B-swizzled, as the out tensor map expects) in the free
-          // Aop region, stored by TMA after the phase-8 barrier
+          // K^ lo region, stored by TMA after the phase-8 barrier
           // (lanes i and i ^ 1 swap one value per token pair and write two adjacent columns)
           const bool odd = lane & 1;
 #pragma unroll
