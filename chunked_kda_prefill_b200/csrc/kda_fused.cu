@@ -448,37 +448,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(sbase + SM_BAR + 8u * (gi & 1), (gi >> 1) & 1u, kWaitLimit)) fail();
       // g_act * log2(e) = lb log2(e) / (1 + 2^(-log2(e) e^A_log (g_raw + dt_bias)))
       const float ca = -a_h * kLog2e;
-      float G[4][4];
+      // rows 4 grp .. 4 grp + 3; warp 0 issues the MMAs this overlaps, so warp 4 (the same SM
+      // sub-partition) takes its rows as well
+      auto group = [&](int grp) {
+        float G[4][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = r0 + i;
-        float gv[4];
-        unpack4(*reinterpret_cast<const uint2*>(sg_tile + atom_off(QGV_ATOM, r, j0)), gv);
+        for (int i = 0; i < 4; ++i) {
+          const int r = 4 * grp + i;
+          float gv[4];
+          unpack4(*reinterpret_cast<const uint2*>(sg_tile + atom_off(QGV_ATOM, r, j0)), gv);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float sgm = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
-          G[i][e] = (r < nn) ? sgm : 0.0f;
+          for (int e = 0; e < 4; ++e) {
+            const float sgm = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
+            G[i][e] = (r < nn) ? sgm : 0.0f;
+          }
         }
-      }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (i > 0)
+        for (int i = 0; i < 4; ++i) {
+          if (i > 0)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) G[i][e] += G[i - 1][e];
-        *reinterpret_cast<float4*>(gtile + (r0 + i) * kD + j0) =
-            make_float4(G[i][0], G[i][1], G[i][2], G[i][3]);
-      }
-      *reinterpret_cast<float4*>(wtot + warp * kD + j0) =
-          make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
-      if (tid < kChunk)
-        beta_s[tid] = (tid < nn) ? __fdividef(1.0f, 1.0f + __expf(-__bfloat162float(blog))) : 0.0f;
+            for (int e = 0; e < 4; ++e) G[i][e] += G[i - 1][e];
+          *reinterpret_cast<float4*>(gtile + (4 * grp + i) * kD + j0) =
+              make_float4(G[i][0], G[i][1], G[i][2], G[i][3]);
+        }
+        *reinterpret_cast<float4*>(wtot + grp * kD + j0) =
+            make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+      };
+      if (warp != 0) group(warp);
+      if (warp == 4) group(0);
+      if (tid >= kChunk && tid < 2 * kChunk)  // (beta: threads 64-127, not warp 0)
+        beta_s[tid - kChunk] =
+            (tid - kChunk < nn) ? __fdividef(1.0f, 1.0f + __expf(-__bfloat162float(blog))) : 0.0f;
     };
-    // Column tid (< 128): exclusive prefix of the 16 warp totals (in place); the block reference
-    // rows (G at rows 15, 31, 47, 63) and from them the per-block constants of the
-    // factorisation; 2^G_last.  Runs under the previous chunk's phase-7 MMAs (after the first).
+    // Column j (threads 128-255, clear of the MMA-issuing warp 0): exclusive prefix of the 16
+    // warp totals (in place); the block reference rows (G at rows 15, 31, 47, 63) and from them
+    // the per-block constants of the factorisation; 2^G_last.  Runs under the previous chunk's
+    // phase-7 MMAs (after an item's first chunk).
     auto front_scan = [&]() {
-      if (tid >= kD) return;
-      const int j = tid;
+      if (tid < kD || tid >= 2 * kD) return;
+      const int j = tid - kD;
       float run = 0.f, ref[4];
 #pragma unroll
       for (int w2 = 0; w2 < 16; ++w2) {
@@ -504,11 +512,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // beta logits (row tid): the item's first chunk now, each later chunk one chunk ahead
     __nv_bfloat16 bl_next = __float2bfloat16_rn(0.f);
+    const bool beta_thread = tid >= kChunk && tid < 2 * kChunk;  // row tid - 64
     {
-      const int t = it.c_begin * kChunk + tid;
+      const int t = it.c_begin * kChunk + tid - kChunk;
       __nv_bfloat16 bl_first = __float2bfloat16_rn(0.f);
-      if (tid < kChunk && t < L) bl_first = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t)];
-      if (tid < kChunk && t + kChunk < L)
+      if (beta_thread && t < L) bl_first = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t)];
+      if (beta_thread && t + kChunk < L)
         bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t + kChunk)];
       front_gate(it.c_begin, gidx, bl_first);
       __syncthreads();
@@ -966,27 +975,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_mma);
       }
       {
-        // the state decay for this chunk (the phase-5 MMAs read the bf16 copies, not TC_S)
-        uint32_t v[16], w2[16];
-        const int col = wg * 32;
-        tmem_ld16(tl + TC_S + col, v);
-        tmem_ld16(tl + TC_S + col + 16, w2);
-        tmem_wait_ld();
+        // the state decay for this chunk (the phase-5 MMAs read the bf16 copies, not TC_S); warp 0
+        // issues the MMAs it overlaps, so warp 4 (same TMEM lanes) takes its columns as well
+        auto decay = [&](int col) {
+          uint32_t v[16], w2[16];
+          tmem_ld16(tl + TC_S + col, v);
+          tmem_ld16(tl + TC_S + col + 16, w2);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e4 = 0; e4 < 16; e4 += 4) {
-          const float4 ga = *reinterpret_cast<const float4*>(gcs + col + e4);
-          const float4 gb = *reinterpret_cast<const float4*>(gcs + col + 16 + e4);
-          v[e4] = __float_as_uint(__uint_as_float(v[e4]) * ga.x);
-          v[e4 + 1] = __float_as_uint(__uint_as_float(v[e4 + 1]) * ga.y);
-          v[e4 + 2] = __float_as_uint(__uint_as_float(v[e4 + 2]) * ga.z);
-          v[e4 + 3] = __float_as_uint(__uint_as_float(v[e4 + 3]) * ga.w);
-          w2[e4] = __float_as_uint(__uint_as_float(w2[e4]) * gb.x);
-          w2[e4 + 1] = __float_as_uint(__uint_as_float(w2[e4 + 1]) * gb.y);
-          w2[e4 + 2] = __float_as_uint(__uint_as_float(w2[e4 + 2]) * gb.z);
-          w2[e4 + 3] = __float_as_uint(__uint_as_float(w2[e4 + 3]) * gb.w);
-        }
-        tmem_st16(tl + TC_S + col, v);
-        tmem_st16(tl + TC_S + col + 16, w2);
+          for (int e4 = 0; e4 < 16; e4 += 4) {
+            const float4 ga = *reinterpret_cast<const float4*>(gcs + col + e4);
+            const float4 gb = *reinterpret_cast<const float4*>(gcs + col + 16 + e4);
+            v[e4] = __float_as_uint(__uint_as_float(v[e4]) * ga.x);
+            v[e4 + 1] = __float_as_uint(__uint_as_float(v[e4 + 1]) * ga.y);
+            v[e4 + 2] = __float_as_uint(__uint_as_float(v[e4 + 2]) * ga.z);
+            v[e4 + 3] = __float_as_uint(__uint_as_float(v[e4 + 3]) * ga.w);
+            w2[e4] = __float_as_uint(__uint_as_float(w2[e4]) * gb.x);
+            w2[e4 + 1] = __float_as_uint(__uint_as_float(w2[e4 + 1]) * gb.y);
+            w2[e4 + 2] = __float_as_uint(__uint_as_float(w2[e4 + 2]) * gb.z);
+            w2[e4 + 3] = __float_as_uint(__uint_as_float(w2[e4 + 3]) * gb.w);
+          }
+          tmem_st16(tl + TC_S + col, v);
+          tmem_st16(tl + TC_S + col + 16, w2);
+        };
+        if (warp != 0) decay(wg * 32);
+        if (warp == 4) decay(0);
         tmem_wait_st();
       }
       wait_mma();
@@ -1069,8 +1082,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (c + 1 < it.c_end) {
         // the next chunk's gate and cumsum under these MMAs, then its successor's beta load
         front_gate(c + 1, gidx + 1, bl_next);
-        const int t2 = t0 + 2 * kChunk + tid;
-        if (c + 2 < it.c_end && tid < kChunk && t2 < L)
+        const int t2 = t0 + 2 * kChunk + tid - kChunk;
+        if (c + 2 < it.c_end && beta_thread && t2 < L)
           bl_next = p.beta[beta_offset(p.layout, p.Nv, p.S, b, h, tok0, t2)];
       }
       wait_mma();
