@@ -390,6 +390,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // phase-1 thread map: warp w owns rows 4w..4w+3 (16-row block w/4), lane owns columns 4l..4l+3
   const int r0 = 4 * warp, j0 = 4 * lane, Jb = warp >> 2;
+  // Byte offset of (row r0 + i, columns j0..j0+3) inside a 64-column atom.  The 128-byte swizzle
+  // depends only on the row mod 8, so the same offset serves every tile whose rows start at a
+  // multiple of 8 (the slot tiles, Aop rows r and 64 + r, the B staircase blocks, K^ lo); a tile
+  // adds its base and, for columns 64-127 (lanes 16-31), its atom stride.
+  uint32_t io[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t r = (uint32_t)(r0 + i);
+    io[i] = r * 128u + (((((uint32_t)j0 & 63u) >> 3) ^ (r & 7u)) << 4) + ((uint32_t)j0 & 7u) * 2u;
+  }
+  const uint32_t colhalf = (uint32_t)(j0 >> 6);
 
   for (int ii = blockIdx.x; ii < p.n_items && !aborted; ii += G_stride) {
     const Item it = item_of(p, ii);
@@ -456,7 +467,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const int r = 4 * grp + i;
           float gv[4];
-          unpack4(*reinterpret_cast<const uint2*>(sg_tile + atom_off(QGV_ATOM, r, j0)), gv);
+          // (row 4 grp + i has the swizzle of row r0 + i: grp and warp have the same parity)
+          const int off = (int)(colhalf * QGV_ATOM + io[i]) + (grp - warp) * 512;
+          unpack4(*reinterpret_cast<const uint2*>(sg_tile + off), gv);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float sgm = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
@@ -569,8 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float qv[4], kv[4];
           const bool valid = r0 + i < n;
           const uint2 zero2 = make_uint2(0u, 0u);
-          const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r0 + i, j0));
-          const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r0 + i, j0));
+          const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]);
+          const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]);
           unpack4(valid ? qw : zero2, qv);
           unpack4(valid ? kw : zero2, kv);
           float ssq = 0.f, ssk = 0.f;
@@ -595,8 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool valid = r < n;
           // rows past the valid length (whatever the storage holds there) become exact zeros
           const uint2 zero2 = make_uint2(0u, 0u);
-          const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j0));
-          const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0));
+          const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]);
+          const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]);
           float qv[4], kv[4];
           unpack4(valid ? qw : zero2, qv);
           unpack4(valid ? kw : zero2, kv);
@@ -622,24 +635,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint2 khp = pack4(kh[0], kh[1], kh[2], kh[3]);
           khlo[i] = make_uint2(split_lo(kh[0], kh[1], khp.x), split_lo(kh[2], kh[3], khp.y));
-          *reinterpret_cast<uint2*>(sm + SM_AOP + sw128_offset(128, r, j0)) = pack4(ka[0], ka[1], ka[2], ka[3]);
-          *reinterpret_cast<uint2*>(sm + SM_AOP + sw128_offset(128, 64 + r, j0)) = pack4(qa[0], qa[1], qa[2], qa[3]);
-          *reinterpret_cast<uint2*>(sq + OFF_Q + atom_off(QGV_ATOM, r, j0)) = pack4(qt[0], qt[1], qt[2], qt[3]);
-          *reinterpret_cast<uint2*>(sq + OFF_K + atom_off(K_ATOM, r, j0)) = khp;
-          *reinterpret_cast<uint2*>(sq + OFF_G + atom_off(QGV_ATOM, r, j0)) = pack4(kt[0], kt[1], kt[2], kt[3]);
-          *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb) + r, j0)) =
+          uint8_t* aop = sm + SM_AOP + colhalf * 16384u + io[i];
+          uint8_t* bst = sm + SM_BT + colhalf * (BT_ROWS * 128u) + io[i];
+          *reinterpret_cast<uint2*>(aop) = pack4(ka[0], ka[1], ka[2], ka[3]);
+          *reinterpret_cast<uint2*>(aop + 8192) = pack4(qa[0], qa[1], qa[2], qa[3]);
+          *reinterpret_cast<uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]) = pack4(qt[0], qt[1], qt[2], qt[3]);
+          *reinterpret_cast<uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]) = khp;
+          *reinterpret_cast<uint2*>(sq + OFF_G + colhalf * QGV_ATOM + io[i]) = pack4(kt[0], kt[1], kt[2], kt[3]);
+          *reinterpret_cast<uint2*>(bst + dcol(Jb) * 128u) =
               pack4(b0[0], b0[1], b0[2], b0[3]);
           if (Jb + 1 <= 3)
-            *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 1) + r, j0)) =
+            *reinterpret_cast<uint2*>(bst + dcol(Jb + 1) * 128u) =
                 pack4(b1[0], b1[1], b1[2], b1[3]);
           if (Jb + 2 <= 3)
-            *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 2) + r, j0)) =
+            *reinterpret_cast<uint2*>(bst + dcol(Jb + 2) * 128u) =
                 pack4(b2[0], b2[1], b2[2], b2[3]);
           if (Jb + 3 <= 3)
-            *reinterpret_cast<uint2*>(sm + SM_BT + sw128_offset(BT_ROWS, dcol(Jb + 3) + r, j0)) =
+            *reinterpret_cast<uint2*>(bst + dcol(Jb + 3) * 128u) =
                 pack4(b3[0], b3[1], b3[2], b3[3]);
           if (!valid || it.zero_v)  // an M run treats v as zero
-            *reinterpret_cast<uint2*>(sq + OFF_V + atom_off(QGV_ATOM, r, j0)) = make_uint2(0, 0);
+            *reinterpret_cast<uint2*>(sq + OFF_V + colhalf * QGV_ATOM + io[i]) = make_uint2(0, 0);
         }
       }
       if (st_thread) tma_store_wait_read();  // the previous out tile (in the K^ lo region) was read
@@ -672,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<uint2*>(sm + SM_KLO + sw128_offset(64, r0 + i, j0)) = khlo[i];
+        *reinterpret_cast<uint2*>(sm + SM_KLO + colhalf * 8192u + io[i]) = khlo[i];
 
       // =================== phase 3: T, Aqk, solve ===================
       // fp32 scratch in the B-tile region (free once the intra MMA has completed)
