@@ -577,6 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint2 khlo[4];  // K^ lo parts of this thread's rows, stored once the intra MMA is done
       {
         float rqv[4], rkv[4];
+        uint2 qwv[4], kwv[4];  // raw q/k words, kept for the operand pass
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float qv[4], kv[4];
@@ -584,8 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint2 zero2 = make_uint2(0u, 0u);
           const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]);
           const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]);
-          unpack4(valid ? qw : zero2, qv);
-          unpack4(valid ? kw : zero2, kv);
+          qwv[i] = valid ? qw : zero2;
+          kwv[i] = valid ? kw : zero2;
+          unpack4(qwv[i], qv);
+          unpack4(kwv[i], kv);
           float ssq = 0.f, ssk = 0.f;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -595,24 +598,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           rqv[i] = ssq;
           rkv[i] = ssk;
         }
+        {
+          // reduce-scatter the 8 partial sums over the warp, then broadcast the 8 totals
+          const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4;
+          float w4[4], x2[2];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            rqv[i] += __shfl_xor_sync(0xffffffffu, rqv[i], o);
-            rkv[i] += __shfl_xor_sync(0xffffffffu, rkv[i], o);
+          for (int k = 0; k < 4; ++k) {
+            const float send = u16 ? rqv[k] : rkv[k];
+            const float keep = u16 ? rkv[k] : rqv[k];
+            w4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
           }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const float send = u8 ? w4[k] : w4[2 + k];
+            const float keep = u8 ? w4[2 + k] : w4[k];
+            x2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+          }
+          float y = (u4 ? x2[1] : x2[0]) + __shfl_xor_sync(0xffffffffu, u4 ? x2[0] : x2[1], 4);
+          y += __shfl_xor_sync(0xffffffffu, y, 2);
+          y += __shfl_xor_sync(0xffffffffu, y, 1);
+          // lane l holds the total of value (l >> 2) & 7: index k + 2 (u8) + 4 (u16) of rq (0-3), rk (4-7)
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            rqv[m] = __shfl_sync(0xffffffffu, y, 4 * (m & 1) + 8 * (m >> 1));
+            rkv[m] = __shfl_sync(0xffffffffu, y, 16 + 4 * (m & 1) + 8 * (m >> 1));
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = r0 + i;
           const bool valid = r < n;
-          // rows past the valid length (whatever the storage holds there) become exact zeros
-          const uint2 zero2 = make_uint2(0u, 0u);
-          const uint2 qw = *reinterpret_cast<const uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]);
-          const uint2 kw = *reinterpret_cast<const uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]);
           float qv[4], kv[4];
-          unpack4(valid ? qw : zero2, qv);
-          unpack4(valid ? kw : zero2, kv);
+          unpack4(qwv[i], qv);
+          unpack4(kwv[i], kv);
           const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
           const float rk = rsqrtf(rkv[i] + 1e-6f);
           float ka[4], qa[4], kt[4], qt[4], kh[4], b0[4], b1[4], b2[4], b3[4];
