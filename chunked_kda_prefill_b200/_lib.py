@@ -5,7 +5,9 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libkda.so")
+# KDA_LIB selects another build of the library (a variant from `build --define`); the default is
+# the in-tree libkda.so.
+LIB_PATH = os.environ.get("KDA_LIB") or os.path.join(PKG, "libkda.so")
 
 # Every symbol include/kda.h declares.
 EXPORTS = ("kda_status_string", "kda_plan_size", "kda_plan", "kda_workspace_size",

@@ -1,10 +1,14 @@
 """Build libkda.so in-tree with nvcc for sm_100a.
 
-    python -m chunked_kda_prefill_b200.build [--force]
+    python -m chunked_kda_prefill_b200.build [--force] [--define NAME=VALUE ...]
 
 Compiles every ``csrc/*.cu`` and ``csrc/*.cpp`` to objects under ``_build/`` (in parallel)
 and links ``chunked_kda_prefill_b200/libkda.so`` with the CUDA runtime linked statically, so
 the library loads on a machine without a GPU (its host entry points work there).
+
+``--define`` builds a variant instead (for example ``KDA_SOLVE_L1=1``, a first-level solve
+variant of the ablation): objects under ``_build_<tag>/`` and ``libkda_<tag>.so``, where
+``<tag>`` joins the definitions; load it with ``KDA_LIB=<path>``.
 """
 from __future__ import annotations
 
@@ -40,11 +44,11 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, verbose):
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src, verbose, build_dir=BUILD, defines=()):
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     if not _stale(obj, [src] + _headers()):
         return obj
-    cmd = [NVCC] + ARCH + COMMON + ["-c", src, "-o", obj + ".tmp"]
+    cmd = [NVCC] + ARCH + COMMON + [f"-D{d}" for d in defines] + ["-c", src, "-o", obj + ".tmp"]
     if src.endswith(".cu") and verbose:
         cmd += ["-Xptxas", "-v"]
     if src.endswith(".cpp"):
@@ -58,26 +62,39 @@ def _compile(src, verbose):
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def variant_tag(defines) -> str:
+    return "_".join(d.replace("=", "").lower() for d in sorted(defines))
+
+
+def build(force: bool = False, verbose: bool = False, defines=()) -> str:
+    defines = tuple(defines)
+    build_dir = BUILD if not defines else BUILD + "_" + variant_tag(defines)
+    lib = LIB if not defines else os.path.join(PKG, f"libkda_{variant_tag(defines)}.so")
+    os.makedirs(build_dir, exist_ok=True)
     srcs = _sources()
     if force:
-        for f in glob.glob(os.path.join(BUILD, "*.o")):
+        for f in glob.glob(os.path.join(build_dir, "*.o")):
             os.remove(f)
     with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    if force or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, verbose, build_dir, defines), srcs))
+    if force or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         # no -lcuda: driver entry points are resolved at run time through the runtime, so
         # the library also loads on a host without the driver
         cmd = [NVCC] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    import argparse
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--define", action="append", default=[])
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.verbose, defines=a.define))

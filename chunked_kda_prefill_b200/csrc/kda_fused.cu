@@ -44,6 +44,13 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 512;
+
+// Variants of the first level of the triangular solve, for the solve ablation (build with
+// -DKDA_SOLVE_L1=n): 0 = 8x8 diagonal inverses + 8->16 merges, CTA-wide (default, fastest);
+// 1 = 16x16 column substitution; 2 = 8x8 + merge warp-local.
+#ifndef KDA_SOLVE_L1
+#define KDA_SOLVE_L1 0
+#endif
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kWaitLimit = 1u << 26;
 
@@ -771,6 +778,95 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncthreads();
       KDA_TS(13);
+#if KDA_SOLVE_L1 == 1
+      // level 1 (variant 1): the 16x16 diagonal inverses by column forward substitution, one
+      // thread per (block, column); two merge levels follow
+      if (tid < 64) {
+        const int I = tid >> 4, cc = tid & 15, base = 16 * I;
+        float x[16];
+        x[0] = (cc == 0) ? 1.f : 0.f;
+#pragma unroll
+        for (int rr = 1; rr < 16; ++rr) {
+          const float* trow = Ts + (base + rr) * TP + base;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int k0 = 0; k0 < rr; k0 += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
+            const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
+          }
+          const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) Xs[(base + k) * TP + base + cc] = x[k];
+      }
+      __syncthreads();
+      KDA_TS(14);
+#elif KDA_SOLVE_L1 == 2
+      // level 1 (variant 2): 8x8 inverses and their 8->16 merge warp-local, one warp per 16x16
+      // block (warps 0, 4, 8, 12), synchronised within the warp only
+      if ((warp & 3) == 0) {
+        const int I = wg;
+        if (lane < 16) {
+          const int base = 16 * I + 8 * (lane >> 3), cc = lane & 7;
+          float x[8];
+          x[0] = (cc == 0) ? 1.f : 0.f;
+#pragma unroll
+          for (int rr = 1; rr < 8; ++rr) {
+            const float* trow = Ts + (base + rr) * TP + base;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k0 = 0; k0 < rr; k0 += 4) {
+              const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
+              const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
+            }
+            const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) Xs[(base + k) * TP + base + cc] = x[k];
+        }
+        __syncwarp();
+        const int rr = lane >> 2, cb = (lane & 3) * 2;
+        const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
+        {
+          const float4 ta = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1);
+          const float4 tb = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1 + 4);
+          const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+          float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float2 xv = *reinterpret_cast<const float2*>(Xs + (c1 + k) * TP + c1 + cb);
+            y0 = fmaf(tv[k], xv.x, y0);
+            y1 = fmaf(tv[k], xv.y, y1);
+          }
+          *reinterpret_cast<float2*>(Ys + (8 * I + rr) * YP + cb) = make_float2(y0, y1);
+        }
+        __syncwarp();
+        {
+          const float4 xa = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 8);
+          const float4 xb = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 12);
+          const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+          float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float2 yv = *reinterpret_cast<const float2*>(Ys + (8 * I + k) * YP + cb);
+            z0 = fmaf(xv[k], yv.x, z0);
+            z1 = fmaf(xv[k], yv.y, z1);
+          }
+          *reinterpret_cast<float2*>(Xs + r1 * TP + c1 + cb) = make_float2(-z0, -z1);
+        }
+      }
+      __syncthreads();
+      KDA_TS(14);
+#else
+      // level 1 (default): 8x8 inverses, then the 8->16 merges, CTA-wide
       // level 1a: X_mm = (I + T_mm)^-1 for the eight 8x8 diagonal blocks; thread = (block, column),
       // rows by forward substitution as dot products over the already final entries
       if (tid < 64) {
@@ -823,6 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncthreads();
       KDA_TS(14);
+#endif
       // level 2: X_{I,I-1} = -X_II T_{I,I-1} X_{I-1,I-1} for I = 1, 3 (two 16x16 merges).  A thread
       // owns a 2x2 output tile and a quarter of the inner dimension; the quarters meet by shuffles.
       {
