@@ -182,9 +182,9 @@ extern "C" __attribute__((visibility("default"))) kda_status_t kda_simt_workspac
 }
 
 // The fused path with every chunk's intermediates (W, U, Q~, K^, Aqk, gamma_last; fp32, the
-// two-kernel workspace layout after its 256-byte header) written to `dump` (if not NULL), and
-// CTA 0's clock64() at each phase boundary of its first 64 chunks written to `tprof` (if not
-// NULL; 16 words per chunk).
+// two-kernel workspace layout after its 256-byte header) written to `dump` (if not NULL).  In a
+// library built with -DKDA_PHASE_TIMING=1, CTA 0 also writes clock64() at each phase boundary of
+// its first 64 chunks to `tprof` (32 words per chunk, if not NULL); the default build ignores it.
 extern "C" __attribute__((visibility("default"))) kda_status_t kda_forward_debug(
     const kda_shape_t* shape, const int32_t* plan_host, const int32_t* plan_dev, size_t n_int32,
     const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,

@@ -99,11 +99,22 @@ constexpr size_t kFusedSmemBytes = SM_END + 1024;
 // per-(block, column) constants of the operand factorisation, indices into SM_CST
 enum : int { CST_REF = 0, CST_GE, CST_P2REF, CST_KFAC, CST_CDIAG, CST_C2, CST_C3, CST_N };
 
-// Phase timestamps for performance analysis (CTA 0, thread 0, first 64 chunks).
+// Phase timestamps for performance analysis (CTA 0, thread 0, first 64 chunks), compiled in
+// only for a profiling build (-DKDA_PHASE_TIMING=1): every thread would otherwise evaluate the
+// check at each of the ~20 phase boundaries of every chunk.
+#ifndef KDA_PHASE_TIMING
+#define KDA_PHASE_TIMING 0
+#endif
+#if KDA_PHASE_TIMING
 #define KDA_TS(slot_)                                                        \
   do {                                                                       \
     if (tprof_on) p.tprof[(size_t)gidx * 32 + (slot_)] = clock64();          \
   } while (0)
+#else
+#define KDA_TS(slot_) \
+  do {                \
+  } while (0)
+#endif
 
 __device__ __forceinline__ uint32_t dcol(int I) { return 8u * I * (I + 1); }
 
@@ -552,7 +563,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t0 = c * kChunk;
       const int n = min(kChunk, L - t0);
       const bool last = (c == it.c_end - 1);
+#if KDA_PHASE_TIMING
       const bool tprof_on = p.tprof && blockIdx.x == 0 && tid == 0 && gidx < 64;
+#endif
       KDA_TS(0);
 
       // =================== phase 1: operand tiles ===================
