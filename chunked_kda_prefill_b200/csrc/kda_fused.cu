@@ -32,6 +32,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "kda_internal.h"
 #include "kda_layout.cuh"
 #include "kda_sm100.cuh"
@@ -644,55 +646,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             rkv[m] = __shfl_sync(0xffffffffu, y, 16 + 4 * (m & 1) + 8 * (m >> 1));
           }
         }
+        // the rows of this warp's 16-row block JB (warp-uniform) as a compile-time constant, so
+        // the staircase copies B^(JB..3) need no runtime block arithmetic or branches
+        auto rows = [&](auto jb_const) {
+          constexpr int JB = decltype(jb_const)::value;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = r0 + i;
-          const bool valid = r < n;
-          float qv[4], kv[4];
-          unpack4(qwv[i], qv);
-          unpack4(kwv[i], kv);
-          const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
-          const float rk = rsqrtf(rkv[i] + 1e-6f);
-          float ka[4], qa[4], kt[4], qt[4], kh[4], b0[4], b1[4], b2[4], b3[4];
+          for (int i = 0; i < 4; ++i) {
+            const int r = r0 + i;
+            const bool valid = r < n;
+            float qv[4], kv[4];
+            unpack4(qwv[i], qv);
+            unpack4(kwv[i], kv);
+            const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
+            const float rk = rsqrtf(rkv[i] + 1e-6f);
+            float ka[4], qa[4], kt[4], qt[4], kh[4], b0[4], b1[4], b2[4], b3[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float Gv = G[i][e];
-            const float kn = kv[e] * rk;
-            const float qn = qv[e] * rq;
-            const float fA = ex2(Gv - k4[CST_REF][e]);
-            const float kbe = kn * ex2(k4[CST_GE][e] - Gv);
-            ka[e] = kn * fA;
-            qa[e] = qn * fA;
-            kt[e] = ka[e] * k4[CST_P2REF][e];
-            qt[e] = qa[e] * k4[CST_P2REF][e];
-            kh[e] = kbe * k4[CST_KFAC][e];
-            b0[e] = kbe * k4[CST_CDIAG][e];  // B^(Jb): diagonal block
-            b1[e] = kbe;                     // B^(Jb+1): reference row is this block's last row
-            b2[e] = kbe * k4[CST_C2][e];     // B^(Jb+2)
-            b3[e] = kbe * k4[CST_C3][e];     // B^(Jb+3)
+            for (int e = 0; e < 4; ++e) {
+              const float Gv = G[i][e];
+              const float kn = kv[e] * rk;
+              const float qn = qv[e] * rq;
+              const float fA = ex2(Gv - k4[CST_REF][e]);
+              const float kbe = kn * ex2(k4[CST_GE][e] - Gv);
+              ka[e] = kn * fA;
+              qa[e] = qn * fA;
+              kt[e] = ka[e] * k4[CST_P2REF][e];
+              qt[e] = qa[e] * k4[CST_P2REF][e];
+              kh[e] = kbe * k4[CST_KFAC][e];
+              b0[e] = kbe * k4[CST_CDIAG][e];  // B^(Jb): diagonal block
+              b1[e] = kbe;                     // B^(Jb+1): reference row is this block's last row
+              if (JB + 2 <= 3) b2[e] = kbe * k4[CST_C2][e];  // B^(Jb+2)
+              if (JB + 3 <= 3) b3[e] = kbe * k4[CST_C3][e];  // B^(Jb+3)
+            }
+            const uint2 khp = pack4(kh[0], kh[1], kh[2], kh[3]);
+            khlo[i] = make_uint2(split_lo(kh[0], kh[1], khp.x), split_lo(kh[2], kh[3], khp.y));
+            uint8_t* aop = sm + SM_AOP + colhalf * 16384u + io[i];
+            uint8_t* bst = sm + SM_BT + colhalf * (BT_ROWS * 128u) + io[i];
+            *reinterpret_cast<uint2*>(aop) = pack4(ka[0], ka[1], ka[2], ka[3]);
+            *reinterpret_cast<uint2*>(aop + 8192) = pack4(qa[0], qa[1], qa[2], qa[3]);
+            *reinterpret_cast<uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]) = pack4(qt[0], qt[1], qt[2], qt[3]);
+            *reinterpret_cast<uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]) = khp;
+            *reinterpret_cast<uint2*>(sq + OFF_G + colhalf * QGV_ATOM + io[i]) = pack4(kt[0], kt[1], kt[2], kt[3]);
+            *reinterpret_cast<uint2*>(bst + dcol(JB) * 128u) =
+                pack4(b0[0], b0[1], b0[2], b0[3]);
+            if (JB + 1 <= 3)
+              *reinterpret_cast<uint2*>(bst + dcol(JB + 1) * 128u) =
+                  pack4(b1[0], b1[1], b1[2], b1[3]);
+            if (JB + 2 <= 3)
+              *reinterpret_cast<uint2*>(bst + dcol(JB + 2) * 128u) =
+                  pack4(b2[0], b2[1], b2[2], b2[3]);
+            if (JB + 3 <= 3)
+              *reinterpret_cast<uint2*>(bst + dcol(JB + 3) * 128u) =
+                  pack4(b3[0], b3[1], b3[2], b3[3]);
+            if (!valid || it.zero_v)  // an M run treats v as zero
+              *reinterpret_cast<uint2*>(sq + OFF_V + colhalf * QGV_ATOM + io[i]) = make_uint2(0, 0);
           }
-          const uint2 khp = pack4(kh[0], kh[1], kh[2], kh[3]);
-          khlo[i] = make_uint2(split_lo(kh[0], kh[1], khp.x), split_lo(kh[2], kh[3], khp.y));
-          uint8_t* aop = sm + SM_AOP + colhalf * 16384u + io[i];
-          uint8_t* bst = sm + SM_BT + colhalf * (BT_ROWS * 128u) + io[i];
-          *reinterpret_cast<uint2*>(aop) = pack4(ka[0], ka[1], ka[2], ka[3]);
-          *reinterpret_cast<uint2*>(aop + 8192) = pack4(qa[0], qa[1], qa[2], qa[3]);
-          *reinterpret_cast<uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]) = pack4(qt[0], qt[1], qt[2], qt[3]);
-          *reinterpret_cast<uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]) = khp;
-          *reinterpret_cast<uint2*>(sq + OFF_G + colhalf * QGV_ATOM + io[i]) = pack4(kt[0], kt[1], kt[2], kt[3]);
-          *reinterpret_cast<uint2*>(bst + dcol(Jb) * 128u) =
-              pack4(b0[0], b0[1], b0[2], b0[3]);
-          if (Jb + 1 <= 3)
-            *reinterpret_cast<uint2*>(bst + dcol(Jb + 1) * 128u) =
-                pack4(b1[0], b1[1], b1[2], b1[3]);
-          if (Jb + 2 <= 3)
-            *reinterpret_cast<uint2*>(bst + dcol(Jb + 2) * 128u) =
-                pack4(b2[0], b2[1], b2[2], b2[3]);
-          if (Jb + 3 <= 3)
-            *reinterpret_cast<uint2*>(bst + dcol(Jb + 3) * 128u) =
-                pack4(b3[0], b3[1], b3[2], b3[3]);
-          if (!valid || it.zero_v)  // an M run treats v as zero
-            *reinterpret_cast<uint2*>(sq + OFF_V + colhalf * QGV_ATOM + io[i]) = make_uint2(0, 0);
+        };
+        switch (Jb) {
+          case 0: rows(std::integral_constant<int, 0>{}); break;
+          case 1: rows(std::integral_constant<int, 1>{}); break;
+          case 2: rows(std::integral_constant<int, 2>{}); break;
+          default: rows(std::integral_constant<int, 3>{}); break;
         }
       }
       if (st_thread) tma_store_wait_read();  // the previous out tile (in the K^ lo region) was read
