@@ -91,10 +91,10 @@ constexpr uint32_t SM_OSTG = SM_KLO;  //   next chunk's phase 2: the out tile fo
 constexpr uint32_t SM_AQK = 221184;   // [64][64] bf16 (phases 3-7)
 constexpr uint32_t SM_GC = 229376;    // fp32 [128]: 2^G_last
 constexpr uint32_t SM_BETA = 229888;  // fp32 [64]
-constexpr uint32_t SM_BAR = 230144;   // raw_full[2], mma
-constexpr uint32_t SM_TSLOT = 230168;
-constexpr uint32_t SM_FLAG = 230172;
-constexpr uint32_t SM_PROD = 230176;  // the TMA producer's state (thread 0 only), 128 bytes
+constexpr uint32_t SM_BAR = 230144;   // raw_full[2], mma, mma_u (the U MMAs of phase 4)
+constexpr uint32_t SM_TSLOT = 230176;
+constexpr uint32_t SM_FLAG = 230180;
+constexpr uint32_t SM_PROD = 230184;  // the TMA producer's state (thread 0 only), 120 bytes
 constexpr uint32_t SM_END = 230304;
 constexpr size_t kFusedSmemBytes = SM_END + 1024;
 
@@ -322,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   const uint32_t bar_mma = sbase + SM_BAR + 16;
+  const uint32_t bar_mma_u = sbase + SM_BAR + 24;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_FLAG);
   float* wtot = reinterpret_cast<float*>(sm + SM_WTOT);
   float* cst = reinterpret_cast<float*>(sm + SM_CST);
@@ -333,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(sbase + SM_BAR, 8);  // one arrival per TMA box of the slot
     mbar_init(sbase + SM_BAR + 8, 8);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_mma_u, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -396,7 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   uint32_t gidx = 0;       // chunks consumed by this CTA
-  uint32_t mma_phase = 0;  // parity of the next MMA-barrier completion
+  uint32_t mma_phase = 0;    // parity of the next MMA-barrier completion
+  uint32_t mma_u_phase = 0;  // and of the phase-4 U MMAs' barrier
   bool aborted = false;
 
   auto fail = [&]() {
@@ -1122,13 +1125,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t aw = smem_desc(as + OFF_G + kk * 2048, QGV_ATOM, 1024);
           mma_ss(tbase + TC_W, aw, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc_w, kk > 0);
         }
+        mma_commit(bar_mma);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t av = smem_desc(as + OFF_V + kk * 2048, QGV_ATOM, 1024);
           mma_ss(tbase + TC_U, av, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc_u, kk > 0);
           mma_ss(tbase + TC_U, av, smem_desc(sbase + SM_XSOL + 8192 + kk * 32, 16, 1024), idesc_u, 1);
         }
-        mma_commit(bar_mma);
+        mma_commit(bar_mma_u);  // the U MMAs are waited for only before -W lo overwrites V
       }
       {
         // the state decay for this chunk (the phase-5 MMAs read the bf16 copies, not TC_S); warp 0
@@ -1167,7 +1171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // j ^ 1 swap one value per row pair, so each writes two adjacent columns of one row.
         const int j = wq + lane;
         const bool odd = lane & 1;
-        uint32_t va[16], vb[16];
+        uint32_t va[16], vb[16], wlo[8];
         tmem_ld16(tl + TC_W + 16 * wg, va);
         tmem_ld16(tl + TC_W + 64 + 16 * wg, vb);
         tmem_wait_ld();
@@ -1180,9 +1184,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int r = 16 * wg + 2 * q + (odd ? 1 : 0);
           const uint32_t off = atom_off(QGV_ATOM, r, j & ~1);
           const uint32_t hi = pack_bf16(x0, x1);
-          const uint32_t lo = pack_bf16(x0 - bf16_lo_of(hi), x1 - bf16_hi_of(hi));
-          *reinterpret_cast<uint32_t*>(sq + OFF_G + off) = hi;
-          *reinterpret_cast<uint32_t*>(sq + OFF_V + off) = lo;
+          wlo[q] = pack_bf16(x0 - bf16_lo_of(hi), x1 - bf16_hi_of(hi));
+          *reinterpret_cast<uint32_t*>(sq + OFF_G + off) = hi;  // K~ was read by the W MMAs
+        }
+        // the lo parts go over V, which the U MMAs read: wait for them first
+        if (!mbar_wait_bounded(bar_mma_u, mma_u_phase, kWaitLimit)) fail();
+        mma_u_phase ^= 1u;
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int r = 16 * wg + 2 * q + (odd ? 1 : 0);
+          *reinterpret_cast<uint32_t*>(sq + OFF_V + atom_off(QGV_ATOM, r, j & ~1)) = wlo[q];
         }
       }
       if (dbg && !it.zero_v) {  // per-chunk intermediates in the two-kernel workspace layout (fp32)
