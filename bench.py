@@ -424,6 +424,78 @@ def _max_over_ranks(x, dist, dev):
     return float(t.item())
 
 
+DECODE_METRIC = "KDA decode step token-heads/s per B200 (one token per sequence and value head)"
+
+
+def decode_bytes(B: int, Nqk: int, Nv: int, D: int = 128) -> int:
+    """Unique HBM bytes of one decode step: fp32 state in and out, bf16 q, k (per qk head), v, g,
+    out, beta, and the gate parameters."""
+    units = B * Nv
+    return (units * D * D * 4 * 2 + B * Nqk * D * 2 * 2 + units * D * 2 * 3 + units * 2
+            + Nv * 4 + Nv * D * 4)
+
+
+def run_decode(args, rank, world):
+    """One decode step per (sequence, value head) with the state updated in place."""
+    import torch
+    import chunked_kda_prefill_b200 as kda
+
+    local = _env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, Nqk, Nv, D = args.decode_batch, 32, 32, 128
+    rng = np.random.default_rng(7 + 1000 * rank)
+
+    def bf16(shape):
+        return torch.from_numpy(W.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32))
+                                .view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k = bf16((B, Nqk, D)), bf16((B, Nqk, D))
+    v, g, beta = bf16((B, Nv, D)), bf16((B, Nv, D)), bf16((B, Nv))
+    A_log = torch.from_numpy(rng.standard_normal(Nv).astype(np.float32)).to(dev)
+    dt_bias = torch.from_numpy(rng.standard_normal((Nv, D)).astype(np.float32)).to(dev)
+    state = torch.from_numpy((0.1 * rng.standard_normal((B, Nv, D, D))).astype(np.float32)).to(dev)
+    out = torch.empty_like(v)
+    stream = torch.cuda.Stream(dev)
+
+    def step():
+        kda.decode(q, k, v, g, beta, D ** -0.5, state, A_log, dt_bias, -5.0, out=out,
+                   state_out=state, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(args.steps):
+                step()
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(end) / args.steps
+    units = B * Nv
+    nbytes = decode_bytes(B, Nqk, Nv, D)
+    peak, peak_kind = measured_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    line = {"metric": DECODE_METRIC, "value": world * units / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded N(0,1) bf16 inputs, 0.1 N(0,1) fp32 state)",
+            "config": {"workload": f"decode_{B}x{Nqk}x{Nv}", "B": B, "Nqk": Nqk, "Nv": Nv,
+                       "D": D, "lower_bound": -5.0, "state": "updated in place",
+                       "l2": f"state ({units * D * D * 4 / 1e9:.2f} GB) larger than L2"},
+            "clocks": clk.report(), "gpu_launches": args.steps,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "kda_decode_kernel",
+                         "algorithmic_bytes": nbytes, "kernel_ms": ms,
+                         "peak_source": f"{peak_kind} hbm_gbs"}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -436,6 +508,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode"],
+                    help="prefill (the default, the headline) or the single-token decode step")
+    ap.add_argument("--decode-batch", type=int, default=256)
     ap.add_argument("--segment-chunks", type=int, default=-1,
                     help="schedule: -1 the planner's choice, 0 whole units, n > 0 segments of n "
                          "chunks (chunk-parallel scan)")
@@ -445,6 +520,8 @@ def main():
     world = _env_int("WORLD_SIZE", 1)
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.mode == "decode":
+        return run_decode(args, rank, world)
     return run_ours(args, rank, world)
 
 
