@@ -110,8 +110,8 @@ def algorithmic_bytes(w: W.Workload, with_initial_state: bool) -> int:
 
 
 def algorithmic_flops(w: W.Workload) -> float:
-    """Dense MMA flops of the chunked method per chunk-head (C=64, D=128): 11.62 MFLOP."""
-    per_chunk = 5 * 2 * 64 * 64 * 128 + 3 * 2 * 64 * 128 * 128
+    """Dense MMA flops of the chunked method per chunk-head (C=64): 11.62 MFLOP at D=128."""
+    per_chunk = 5 * 2 * 64 * 64 * w.D + 3 * 2 * 64 * w.D * w.D
     chunks = sum(math.ceil(L / 64) for L in w.lengths) * w.Nv
     return float(per_chunk * chunks)
 

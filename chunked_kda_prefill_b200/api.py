@@ -200,9 +200,9 @@ def decode(q, k, v, g, beta, scale: float, state, A_log, dt_bias, lower_bound: f
            stream: torch.cuda.Stream | None = None):
     """One decode step (one token per sequence) through kda_decode.
 
-    q, k: bf16 [B, Nqk, 128]; v, g: bf16 [B, Nv, 128]; beta: bf16 [B, Nv]; state: fp32
-    [B, Nv, 128, 128] or None (zeros).  Returns (out [B, Nv, 128] bf16, state_out); pass
-    ``state_out=state`` to update the state in place.
+    q, k: bf16 [B, Nqk, D]; v, g: bf16 [B, Nv, D]; beta: bf16 [B, Nv]; state: fp32
+    [B, Nv, D, D] or None (zeros), D = 128 or 64.  Returns (out [B, Nv, D] bf16, state_out);
+    pass ``state_out=state`` to update the state in place.
     """
     dev = q.device
     if dev.type != "cuda":

@@ -56,6 +56,7 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
     return KDA_ERR_NULL;
   st = validate_plan(plan_host, n_int32, shape);
   if (st != KDA_OK) return st;
+  if (path == PATH_SIMT && shape->D != kD) return KDA_ERR_DIM;  // the fp32 path is D = 128 only
   if (!std::isfinite(scale)) return KDA_ERR_LOWER_BOUND;
   if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_LOWER_BOUND;
   {
@@ -72,10 +73,11 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   // aliasing: outputs must not overlap any input or each other
   const long long rows =
       shape->layout == KDA_LAYOUT_TND ? (long long)shape->S : (long long)shape->B * shape->S;
-  const size_t qk_bytes = (size_t)rows * shape->Nqk * kD * 2;
-  const size_t vg_bytes = (size_t)rows * shape->Nv * kD * 2;
+  const size_t D = (size_t)shape->D;
+  const size_t qk_bytes = (size_t)rows * shape->Nqk * D * 2;
+  const size_t vg_bytes = (size_t)rows * shape->Nv * D * 2;
   const size_t beta_bytes = (size_t)rows * shape->Nv * 2;
-  const size_t st_bytes = (size_t)shape->B * shape->Nv * kD * kD * 4;
+  const size_t st_bytes = (size_t)shape->B * shape->Nv * D * D * 4;
   const Range r_out = range_of(out, vg_bytes), r_fs = range_of(final_state, st_bytes);
   const Range ins[] = {range_of(q, qk_bytes), range_of(k, qk_bytes), range_of(v, vg_bytes),
                        range_of(g, vg_bytes), range_of(beta, beta_bytes),
@@ -96,6 +98,7 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   p.Nqk = shape->Nqk;
   p.Nv = shape->Nv;
   p.S = shape->S;
+  p.D = shape->D;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
   p.v = static_cast<const __nv_bfloat16*>(v);

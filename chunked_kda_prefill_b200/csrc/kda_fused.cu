@@ -169,6 +169,7 @@ struct Item {
   int ident;              // start from the identity (M run)
   const float* s_in;      // start state (null: zero; ignored for the identity)
   float* s_out;           // where the final state goes (null: nowhere)
+  int in_ld, out_ld;      // their row length: D for the caller's states, kD for state slots
   int write_out, zero_v, pad;  // write outputs; treat v as zero; zero-fill rows past L
 };
 
@@ -199,7 +200,7 @@ __device__ Item item_of(const Params& p, int i) {
   it.L = rec[PR_LEN];
   it.coff = rec[PR_CHUNK_OFFSET];
   const int nch = rec[PR_CHUNKS];
-  const size_t bh = ((size_t)it.b * p.Nv + it.h) * kD * kD;
+  const size_t bh = ((size_t)it.b * p.Nv + it.h) * p.D * p.D;
   const float* s0 = p.S0 ? p.S0 + bh : nullptr;
   it.ident = 0;
   it.zero_v = 0;
@@ -208,6 +209,7 @@ __device__ Item item_of(const Params& p, int i) {
     it.c_end = nch;
     it.s_in = s0;
     it.s_out = p.Sf + bh;
+    it.in_ld = it.out_ld = p.D;
     it.write_out = 1;
     it.pad = 1;
     return it;
@@ -220,11 +222,14 @@ __device__ Item item_of(const Params& p, int i) {
     sgm = (j + 1) >> 1;
     if (j == 0) {  // the first segment, from the true initial state
       it.s_in = s0;
+      it.in_ld = p.D;
       it.s_out = (nseg == 1) ? p.Sf + bh : slot_ptr(p, base, SLOT_START);
+      it.out_ld = (nseg == 1) ? p.D : kD;
       it.write_out = 1;
       it.pad = (nseg == 1);
     } else {
       it.s_in = nullptr;
+      it.in_ld = it.out_ld = kD;
       it.write_out = 0;
       it.pad = 0;
       if (j & 1) {
@@ -238,7 +243,9 @@ __device__ Item item_of(const Params& p, int i) {
   } else {
     sgm = i - base + 1;
     it.s_in = slot_ptr(p, base + sgm - 1, SLOT_START);
+    it.in_ld = kD;
     it.s_out = (sgm == nseg - 1) ? p.Sf + bh : nullptr;
+    it.out_ld = p.D;
     it.write_out = 1;
     it.pad = (sgm == nseg - 1);
   }
@@ -432,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float lbl2 = p.lower_bound * kLog2e;
     float dtb[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) dtb[e] = p.dt_bias[h * kD + j0 + e];
+    for (int e = 0; e < 4; ++e) dtb[e] = (j0 < p.D) ? p.dt_bias[h * p.D + j0 + e] : 0.f;
 
     // ---- start state (the item's: initial_state, a state slot, zeros or the identity):
     //      fp32 -> TMEM S, bf16 hi/lo -> TMEM state operand ----
@@ -449,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int d = i - (col0 + c);
             x = make_float4(d == 0 ? 1.f : 0.f, d == 1 ? 1.f : 0.f, d == 2 ? 1.f : 0.f,
                             d == 3 ? 1.f : 0.f);
-          } else if (it.s_in) {
-            x = *reinterpret_cast<const float4*>(it.s_in + (size_t)i * kD + col0 + c);
+          } else if (it.s_in && i < it.in_ld && col0 + c < it.in_ld) {
+            x = *reinterpret_cast<const float4*>(it.s_in + (size_t)i * it.in_ld + col0 + c);
           }
           fv[c] = __float_as_uint(x.x);
           fv[c + 1] = __float_as_uint(x.y);
@@ -1329,12 +1336,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // the sequence's last, partial chunk: plain stores of the valid rows
-          const int64_t ostride = (p.layout == KDA_LAYOUT_BNSD) ? kD : (int64_t)p.Nv * kD;
-          __nv_bfloat16* orow = p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t0) + i;
+          const int64_t ostride = (p.layout == KDA_LAYOUT_BNSD) ? p.D : (int64_t)p.Nv * p.D;
+          __nv_bfloat16* orow = p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t0, p.D) + i;
+          if (i < p.D) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int t = 16 * wg + e;
-            if (t < n) orow[t * ostride] = __float2bfloat16_rn(__uint_as_float(vo[e]));
+            for (int e = 0; e < 16; ++e) {
+              const int t = 16 * wg + e;
+              if (t < n) orow[t * ostride] = __float2bfloat16_rn(__uint_as_float(vo[e]));
+            }
           }
         }
         KDA_TS(18);
@@ -1354,8 +1363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(tl + TC_SHI + col / 2, hi);
         tmem_st16(tl + TC_SLO + col / 2, lo);
-        if (last && it.s_out) {
-          float* dst = it.s_out + (size_t)i * kD + col;
+        if (last && it.s_out && i < it.out_ld && col < it.out_ld) {
+          float* dst = it.s_out + (size_t)i * it.out_ld + col;
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
             *reinterpret_cast<float4*>(dst + e) = make_float4(
@@ -1377,8 +1386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const LoadRec ur{b, h, 0, tok0, 0, 0};
         chunk_coords(p, ur, c, qc1, qc2, oc1, oc2);
         const int half = warp - 9;
-        tma_store_3d(&maps.o, sbase + SM_OSTG + half * 8192, 64 * half, oc1, oc2);
-        tma_store_commit();
+        if (64 * half < p.D) {  // (D = 64: the upper half is padding)
+          tma_store_3d(&maps.o, sbase + SM_OSTG + half * 8192, 64 * half, oc1, oc2);
+          tma_store_commit();
+        }
       }
       if (*abort_flag) {
         aborted = true;
@@ -1387,10 +1398,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // rows past the valid length (BNSD/BSND storage padding) are defined as zero
     if (!aborted && it.pad && p.layout != KDA_LAYOUT_TND) {
-      for (int e = tid; e < (p.S - L) * 16; e += kThreads) {
-        const int t = L + (e >> 4), q8 = (e & 15) * 8;
-        *reinterpret_cast<uint4*>(p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t) + q8) =
-            make_uint4(0, 0, 0, 0);
+      const int per_row = p.D / 8;  // 16-byte stores per row
+      for (int e = tid; e < (p.S - L) * per_row; e += kThreads) {
+        const int t = L + e / per_row, q8 = (e % per_row) * 8;
+        *reinterpret_cast<uint4*>(p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t, p.D) +
+                                  q8) = make_uint4(0, 0, 0, 0);
       }
     }
   }
@@ -1413,17 +1425,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 namespace {
 
-bool make_map(CUtensorMap* m, const void* base, int layout, int B, int NX, int S) {
+// D = 64: the kernel still loads two 64-column boxes per tile; the second lies wholly past the
+// tensor's D columns and reads as zeros, so the upper 64 channels of q, k, v, g are zero.
+bool make_map(CUtensorMap* m, const void* base, int layout, int B, int NX, int S, int D) {
   uint64_t dims[3], strides[2];
   uint32_t box[3];
   if (layout == KDA_LAYOUT_BNSD) {
-    dims[0] = kD; dims[1] = (uint64_t)S; dims[2] = (uint64_t)B * NX;
-    strides[0] = kD * 2; strides[1] = (uint64_t)S * kD * 2;
+    dims[0] = (uint64_t)D; dims[1] = (uint64_t)S; dims[2] = (uint64_t)B * NX;
+    strides[0] = (uint64_t)D * 2; strides[1] = (uint64_t)S * D * 2;
     box[0] = 64; box[1] = 64; box[2] = 1;
   } else {
     const uint64_t rows = (layout == KDA_LAYOUT_BSND) ? (uint64_t)B * S : (uint64_t)S;
-    dims[0] = kD; dims[1] = (uint64_t)NX; dims[2] = rows;
-    strides[0] = kD * 2; strides[1] = (uint64_t)NX * kD * 2;
+    dims[0] = (uint64_t)D; dims[1] = (uint64_t)NX; dims[2] = rows;
+    strides[0] = (uint64_t)D * 2; strides[1] = (uint64_t)NX * D * 2;
     box[0] = 64; box[1] = 1; box[2] = 64;
   }
   return encode_bf16_3d(m, base, dims, strides, box);
@@ -1446,11 +1460,11 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
     configured_device = dev;
   }
   Maps m;
-  if (!make_map(&m.q, p.q, p.layout, p.B, p.Nqk, p.S) ||
-      !make_map(&m.k, p.k, p.layout, p.B, p.Nqk, p.S) ||
-      !make_map(&m.v, p.v, p.layout, p.B, p.Nv, p.S) ||
-      !make_map(&m.g, p.g, p.layout, p.B, p.Nv, p.S) ||
-      !make_map(&m.o, p.out, p.layout, p.B, p.Nv, p.S))
+  if (!make_map(&m.q, p.q, p.layout, p.B, p.Nqk, p.S, p.D) ||
+      !make_map(&m.k, p.k, p.layout, p.B, p.Nqk, p.S, p.D) ||
+      !make_map(&m.v, p.v, p.layout, p.B, p.Nv, p.S, p.D) ||
+      !make_map(&m.g, p.g, p.layout, p.B, p.Nv, p.S, p.D) ||
+      !make_map(&m.o, p.out, p.layout, p.B, p.Nv, p.S, p.D))
     return cudaErrorInvalidValue;
   if (p.n_items < 1) return cudaSuccess;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;

@@ -27,14 +27,14 @@ int32_t plan_checksum(const int32_t* plan, size_t n) {
 kda_status_t validate_shape(const kda_shape_t* s) {
   if (!s) return KDA_ERR_NULL;
   if (s->layout < KDA_LAYOUT_BNSD || s->layout > KDA_LAYOUT_TND) return KDA_ERR_LAYOUT;
-  if (s->D != kD) return KDA_ERR_DIM;
+  if (s->D != kD && s->D != 64) return KDA_ERR_DIM;
   if (s->B < 1 || s->S < 1) return KDA_ERR_SHAPE;
   if (s->Nqk < 1 || s->Nv < s->Nqk || s->Nv % s->Nqk != 0) return KDA_ERR_HEADS;
   // index ranges: units fit int32; every tensor's element count fits int64 comfortably
   const long long units = (long long)s->B * s->Nv;
   if (units > INT_MAX / 2) return KDA_ERR_SHAPE;
   const long long rows = (s->layout == KDA_LAYOUT_TND) ? (long long)s->S : (long long)s->B * s->S;
-  if (rows * (long long)s->Nv * kD > (1LL << 46)) return KDA_ERR_SHAPE;
+  if (rows * (long long)s->Nv * s->D > (1LL << 46)) return KDA_ERR_SHAPE;
   return KDA_OK;
 }
 
@@ -85,7 +85,7 @@ extern "C" const char* kda_status_string(kda_status_t st) {
     case KDA_ERR_LAYOUT: return "KDA_ERR_LAYOUT: layout must be BNSD, BSND or TND";
     case KDA_ERR_SHAPE: return "KDA_ERR_SHAPE: B and S must be >= 1 and sizes must fit";
     case KDA_ERR_HEADS: return "KDA_ERR_HEADS: need 1 <= Nqk <= Nv and Nv % Nqk == 0";
-    case KDA_ERR_DIM: return "KDA_ERR_DIM: head dim D must be 128";
+    case KDA_ERR_DIM: return "KDA_ERR_DIM: head dim D must be 64 or 128";
     case KDA_ERR_LOWER_BOUND:
       return "KDA_ERR_LOWER_BOUND: lower_bound must be in [-5, 0] and scale finite";
     case KDA_ERR_SEQLENS: return "KDA_ERR_SEQLENS: cu_seqlens malformed";

@@ -10,6 +10,7 @@ namespace kda {
 
 struct Params {
   int layout, B, Nqk, Nv, S;
+  int D;  // head dim of the tensors (64 or 128); the kernels compute at kD = 128 channels
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
@@ -37,10 +38,10 @@ struct Params {
 // Element offset of the D-vector of (sequence b, head hx of NX heads, token t of the sequence).
 // BNSD [B,NX,S,D], BSND [B,S,NX,D], TND [T,NX,D] with the sequence starting at packed row tok0.
 __device__ __forceinline__ int64_t row_offset(int layout, int NX, int S, int b, int hx, int tok0,
-                                              int t) {
-  if (layout == KDA_LAYOUT_BNSD) return (((int64_t)b * NX + hx) * S + t) * kD;
-  if (layout == KDA_LAYOUT_BSND) return (((int64_t)b * S + t) * NX + hx) * kD;
-  return ((int64_t)(tok0 + t) * NX + hx) * kD;
+                                              int t, int D = kD) {
+  if (layout == KDA_LAYOUT_BNSD) return (((int64_t)b * NX + hx) * S + t) * D;
+  if (layout == KDA_LAYOUT_BSND) return (((int64_t)b * S + t) * NX + hx) * D;
+  return ((int64_t)(tok0 + t) * NX + hx) * D;
 }
 
 // Offset of beta for (b, value head h, token t): BNSD [B,Nv,S], BSND [B,S,Nv], TND [T,Nv].

@@ -53,7 +53,7 @@ typedef enum {
   KDA_ERR_LAYOUT = 2,      /* layout is not BNSD, BSND or TND */
   KDA_ERR_SHAPE = 3,       /* B < 1, S < 1, or a size does not fit the index types */
   KDA_ERR_HEADS = 4,       /* not 1 <= Nqk <= Nv with Nv % Nqk == 0 */
-  KDA_ERR_DIM = 5,         /* D != 128 */
+  KDA_ERR_DIM = 5,         /* D is neither 128 nor 64 */
   KDA_ERR_LOWER_BOUND = 6, /* lower_bound not in [-5, 0], or scale not finite */
   KDA_ERR_SEQLENS = 7,     /* cu_seqlens malformed (see kda_plan) */
   KDA_ERR_PLAN = 8,        /* plan buffer too small, corrupt, or built for another shape */
@@ -79,7 +79,7 @@ typedef struct {
   int32_t Nqk;    /* query/key heads */
   int32_t Nv;     /* value heads; value head h reads q/k head h / (Nv / Nqk) */
   int32_t S;      /* storage length per slot (BNSD/BSND) or total packed tokens T (TND) */
-  int32_t D;      /* head dim, must be 128 (Dk = Dv = D) */
+  int32_t D;      /* head dim, 128 or 64 (Dk = Dv = D); see kda_forward for D = 64 */
 } kda_shape_t;
 
 /* Chunk length of the method (tokens). */
@@ -142,7 +142,13 @@ KDA_API kda_status_t kda_workspace_size(const int32_t* plan_host, size_t n_int32
  *                  even); rows past a sequence's valid length are written as zeros.
  *   final_state  : fp32 [B,Nv,D,D]; must not overlap initial_state.
  * Rows of the inputs past a valid length are never read.  Asynchronous: returns once the
- * kernels are enqueued on `stream`. */
+ * kernels are enqueued on `stream`.
+ * Head dim: the FlashKDA README (约束说明) fixes D = 128; D = 64 is the small-head case that FLA
+ * PR 656 ("[kda] add recursive block intra", its summary and timing table) benchmarks.  A D = 64
+ * problem runs through the same kernels as D = 128 with the upper 64 channels of q, k, v and g
+ * read as zeros (the tensor maps end at D), dt_bias and the states indexed with row length D,
+ * and only the first D output channels stored: zero channels add nothing to the q/k norms,
+ * the scores or the state, so the result is the D = 64 operator, at the cost of a D = 128 one. */
 KDA_API kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* plan_host,
                          const int32_t* plan_dev, size_t n_int32, const void* q, const void* k,
                          const void* v, const void* g, const void* beta, float scale,
@@ -191,7 +197,7 @@ KDA_API kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int32_t
  * with kda_forward's in-op activations (q, k L2-normalised; beta = sigmoid(logit);
  * g = lower_bound * sigmoid(e^A_log[h] (g_raw + dt_bias[h,:]))), one token per sequence.
  *   B, Nqk, Nv, D: sequences, query/key heads, value heads (Nv % Nqk == 0; value head h reads
- *                  query/key head h / (Nv / Nqk)), head dim (must be 128).
+ *                  query/key head h / (Nv / Nqk)), head dim (128 or 64).
  *   q, k         : bf16 [B, Nqk, D];  v, g: bf16 [B, Nv, D];  beta: bf16 [B, Nv] (logits).
  *   scale        : finite;  A_log: fp32 [Nv];  dt_bias: fp32 [Nv, D];  lower_bound in [-5, 0].
  *   state_in     : fp32 [B, Nv, D(Dv), D(Dk)], or NULL for zeros.

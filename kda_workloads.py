@@ -120,7 +120,7 @@ SCALE128 = 1.0 / math.sqrt(128.0)
 
 
 def workload(idx: int) -> Workload:
-    """The five synthetic workloads (1-based index)."""
+    """The five synthetic workloads (1-based index), and 6: the head-dim-64 workload."""
     if idx == 1:
         return Workload("tiny_bnsd_1x1x256", "BNSD", 1, 1, 1, 256, 128, [256], -5.0, SCALE128,
                         "zeros", seed=1)
@@ -137,6 +137,10 @@ def workload(idx: int) -> Workload:
     if idx == 5:
         return Workload("large_bnsd_4x32x16384", "BNSD", 4, 32, 32, 16384, 128, [16384] * 4, -5.0,
                         SCALE128, "zeros", seed=5)
+    if idx == 6:
+        # head dim 64: the largest K = 64 shape of FLA PR 656's timing table (B=8, T=4096, H=32)
+        return Workload("headdim64_bnsd_8x32x4096", "BNSD", 8, 32, 32, 4096, 64, [4096] * 8,
+                        -5.0, 1.0 / math.sqrt(64.0), "zeros", seed=6)
     raise ValueError(idx)
 
 

@@ -56,7 +56,7 @@ def _plan(L, shape, cu=None, sms=148):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(D=64), 5), (dict(B=0), 3), (dict(S=0), 3), (dict(Nqk=0), 4), (dict(Nqk=3, Nv=2), 4),
+    (dict(D=96), 5), (dict(D=256), 5), (dict(D=0), 5), (dict(B=0), 3), (dict(S=0), 3), (dict(Nqk=0), 4), (dict(Nqk=3, Nv=2), 4),
     (dict(Nqk=3, Nv=4), 4), (dict(layout=3), 2), (dict(layout=-1), 2)])
 def test_shape_checks(L, kw, code):
     st, _ = _plan(L, _shape(**kw))
@@ -163,8 +163,20 @@ def _dec(L, B=2, Nqk=1, Nv=2, D=128, **kw):
                         a["s0"], a["A_log"], a["dt"], a["lb"], a["out"], a["s1"], None)
 
 
+def test_head_dim_64_plans(L):
+    # D = 64 runs through the D = 128 kernels (upper channels read as zeros); the plan records D
+    for layout, cu in ((0, None), (1, [0, 100, 256]), (2, [0, 7, 256])):
+        B = 1 if cu is None else len(cu) - 1
+        st, buf = _plan(L, _shape(layout=layout, B=B, Nqk=2, Nv=4, S=256, D=64), cu)
+        assert st == 0, (layout, st)
+        ws = ctypes.c_size_t(0)
+        assert L.kda_workspace_size(buf.ctypes.data_as(P_I32), buf.size, ctypes.byref(ws)) == 0
+        assert ws.value >= 256
+
+
 def test_decode_argument_checks(L):
-    assert _dec(L, D=64) == 5
+    assert _dec(L, D=96) == 5
+    assert _dec(L, D=256) == 5
     assert _dec(L, B=0) == 3
     assert _dec(L, Nv=3, Nqk=2) == 4
     assert _dec(L, q=None) == 1
