@@ -169,7 +169,6 @@ struct Item {
   int ident;              // start from the identity (M run)
   const float* s_in;      // start state (null: zero; ignored for the identity)
   float* s_out;           // where the final state goes (null: nowhere)
-  int in_ld, out_ld;      // their row length: D for the caller's states, kD for state slots
   int write_out, zero_v, pad;  // write outputs; treat v as zero; zero-fill rows past L
 };
 
@@ -178,6 +177,7 @@ __device__ __forceinline__ float* slot_ptr(const Params& p, int slot, int part) 
 }
 
 // Item i of this launch (every argument comes from the plan; see the Item comment).
+template <int DIM>
 __device__ Item item_of(const Params& p, int i) {
   const int32_t* R = p.plan + kPlanHeader;
   int u = i;
@@ -200,7 +200,7 @@ __device__ Item item_of(const Params& p, int i) {
   it.L = rec[PR_LEN];
   it.coff = rec[PR_CHUNK_OFFSET];
   const int nch = rec[PR_CHUNKS];
-  const size_t bh = ((size_t)it.b * p.Nv + it.h) * p.D * p.D;
+  const size_t bh = ((size_t)it.b * p.Nv + it.h) * DIM * DIM;
   const float* s0 = p.S0 ? p.S0 + bh : nullptr;
   it.ident = 0;
   it.zero_v = 0;
@@ -209,7 +209,6 @@ __device__ Item item_of(const Params& p, int i) {
     it.c_end = nch;
     it.s_in = s0;
     it.s_out = p.Sf + bh;
-    it.in_ld = it.out_ld = p.D;
     it.write_out = 1;
     it.pad = 1;
     return it;
@@ -222,14 +221,11 @@ __device__ Item item_of(const Params& p, int i) {
     sgm = (j + 1) >> 1;
     if (j == 0) {  // the first segment, from the true initial state
       it.s_in = s0;
-      it.in_ld = p.D;
       it.s_out = (nseg == 1) ? p.Sf + bh : slot_ptr(p, base, SLOT_START);
-      it.out_ld = (nseg == 1) ? p.D : kD;
       it.write_out = 1;
       it.pad = (nseg == 1);
     } else {
       it.s_in = nullptr;
-      it.in_ld = it.out_ld = kD;
       it.write_out = 0;
       it.pad = 0;
       if (j & 1) {
@@ -243,9 +239,7 @@ __device__ Item item_of(const Params& p, int i) {
   } else {
     sgm = i - base + 1;
     it.s_in = slot_ptr(p, base + sgm - 1, SLOT_START);
-    it.in_ld = kD;
     it.s_out = (sgm == nseg - 1) ? p.Sf + bh : nullptr;
-    it.out_ld = p.D;
     it.write_out = 1;
     it.pad = (sgm == nseg - 1);
   }
@@ -258,10 +252,11 @@ __device__ Item item_of(const Params& p, int i) {
 struct LoadRec {
   int b, h, hq, tok0, c_begin, c_end;
 };
+template <int DIM>
 __device__ __forceinline__ LoadRec load_rec(const Params& p, int i) {
   LoadRec r{0, 0, 0, 0, 0, 0};
   if (i < p.n_items) {
-    const Item it = item_of(p, i);
+    const Item it = item_of<DIM>(p, i);
     r = LoadRec{it.b, it.h, it.hq, it.tok0, it.c_begin, it.c_end};
   }
   return r;
@@ -313,6 +308,9 @@ __device__ __forceinline__ void issue_box(const Params& p, const Maps& m, uint32
 
 }  // namespace
 
+// DIM: the tensors' head dim (128, or 64 with the upper channels zero-filled); every tile,
+// TMEM accumulator and MMA is 128 channels wide either way.
+template <int DIM>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_kernel(const Params p, const __grid_constant__ Maps maps, float* dbg) {
   extern __shared__ uint8_t smem_raw[];
@@ -378,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pr.pu += G_stride;
       pr.cur = pr.next;
       pr.pc = pr.cur.c_begin;
-      pr.next = load_rec(p, pr.pu + G_stride);
+      pr.next = load_rec<DIM>(p, pr.pu + G_stride);
     }
   };
   auto issue_planned = [&](int box) {
@@ -389,9 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     prod->pu = blockIdx.x;
     prod->issued = 0;
-    prod->cur = load_rec(p, blockIdx.x);
+    prod->cur = load_rec<DIM>(p, blockIdx.x);
     prod->pc = prod->cur.c_begin;
-    prod->next = load_rec(p, blockIdx.x + G_stride);
+    prod->next = load_rec<DIM>(p, blockIdx.x + G_stride);
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.k);
     tma_prefetch_desc(&maps.v);
@@ -433,13 +431,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t colhalf = (uint32_t)(j0 >> 6);
 
   for (int ii = blockIdx.x; ii < p.n_items && !aborted; ii += G_stride) {
-    const Item it = item_of(p, ii);
+    const Item it = item_of<DIM>(p, ii);
     const int b = it.b, h = it.h, tok0 = it.tok0, L = it.L, coff = it.coff;
     const float a_h = expf(p.A_log[h]);
     const float lbl2 = p.lower_bound * kLog2e;
     float dtb[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) dtb[e] = (j0 < p.D) ? p.dt_bias[h * p.D + j0 + e] : 0.f;
+    for (int e = 0; e < 4; ++e) dtb[e] = (j0 < DIM) ? p.dt_bias[h * DIM + j0 + e] : 0.f;
 
     // ---- start state (the item's: initial_state, a state slot, zeros or the identity):
     //      fp32 -> TMEM S, bf16 hi/lo -> TMEM state operand ----
@@ -456,8 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int d = i - (col0 + c);
             x = make_float4(d == 0 ? 1.f : 0.f, d == 1 ? 1.f : 0.f, d == 2 ? 1.f : 0.f,
                             d == 3 ? 1.f : 0.f);
-          } else if (it.s_in && i < it.in_ld && col0 + c < it.in_ld) {
-            x = *reinterpret_cast<const float4*>(it.s_in + (size_t)i * it.in_ld + col0 + c);
+          } else if (it.s_in && i < DIM && col0 + c < DIM) {
+            x = *reinterpret_cast<const float4*>(it.s_in + (size_t)i * DIM + col0 + c);
           }
           fv[c] = __float_as_uint(x.x);
           fv[c + 1] = __float_as_uint(x.y);
@@ -1336,9 +1334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // the sequence's last, partial chunk: plain stores of the valid rows
-          const int64_t ostride = (p.layout == KDA_LAYOUT_BNSD) ? p.D : (int64_t)p.Nv * p.D;
-          __nv_bfloat16* orow = p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t0, p.D) + i;
-          if (i < p.D) {
+          const int64_t ostride = (p.layout == KDA_LAYOUT_BNSD) ? DIM : (int64_t)p.Nv * DIM;
+          __nv_bfloat16* orow = p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t0, DIM) + i;
+          if (i < DIM) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int t = 16 * wg + e;
@@ -1363,8 +1361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(tl + TC_SHI + col / 2, hi);
         tmem_st16(tl + TC_SLO + col / 2, lo);
-        if (last && it.s_out && i < it.out_ld && col < it.out_ld) {
-          float* dst = it.s_out + (size_t)i * it.out_ld + col;
+        if (last && it.s_out && i < DIM && col < DIM) {
+          float* dst = it.s_out + (size_t)i * DIM + col;
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
             *reinterpret_cast<float4*>(dst + e) = make_float4(
@@ -1386,7 +1384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const LoadRec ur{b, h, 0, tok0, 0, 0};
         chunk_coords(p, ur, c, qc1, qc2, oc1, oc2);
         const int half = warp - 9;
-        if (64 * half < p.D) {  // (D = 64: the upper half is padding)
+        if (64 * half < DIM) {  // (D = 64: the upper half is padding)
           tma_store_3d(&maps.o, sbase + SM_OSTG + half * 8192, 64 * half, oc1, oc2);
           tma_store_commit();
         }
@@ -1398,10 +1396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // rows past the valid length (BNSD/BSND storage padding) are defined as zero
     if (!aborted && it.pad && p.layout != KDA_LAYOUT_TND) {
-      const int per_row = p.D / 8;  // 16-byte stores per row
+      const int per_row = DIM / 8;  // 16-byte stores per row
       for (int e = tid; e < (p.S - L) * per_row; e += kThreads) {
         const int t = L + e / per_row, q8 = (e % per_row) * 8;
-        *reinterpret_cast<uint4*>(p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t, p.D) +
+        *reinterpret_cast<uint4*>(p.out + row_offset(p.layout, p.Nv, p.S, b, h, tok0, t, DIM) +
                                   q8) = make_uint4(0, 0, 0, 0);
       }
     }
@@ -1452,7 +1450,10 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kda_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(kda_fused_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kFusedSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kda_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kFusedSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1468,7 +1469,8 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   if (p.n_items < 1) return cudaSuccess;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
-  kda_fused_kernel<<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
+  if (p.D == kD) kda_fused_kernel<kD><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
+  else kda_fused_kernel<64><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
   return cudaGetLastError();
 }
 
