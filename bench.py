@@ -7,7 +7,9 @@ A step is one kda_forward over the large prefill (B=4, Nqk=Nv=32, S=16384, D=128
 synthetic bf16 inputs ~ N(0,1)).  Units (sequence, value head) are independent, so N > 1 runs one
 replica of the workload per GPU with no collective on the data path (weak scaling); torchrun
 supplies RANK / LOCAL_RANK / WORLD_SIZE.  ``--impl reference`` times the fp64 CPU oracle on a
-bounded sample of the same workload (rank 0 only).
+bounded sample of the same workload (rank 0 only).  ``--mode decode`` times the single-token
+decode step, ``--mode cp`` context parallelism (one sequence split over the ranks; with one
+process ``--cp-emulate E`` runs E ranks' work one after another).
 """
 from __future__ import annotations
 
@@ -496,6 +498,109 @@ def run_decode(args, rank, world):
     return 0
 
 
+CP_METRIC = "KDA prefill tokens/s, one sequence split over ranks (context parallel)"
+
+
+def run_cp(args, rank, world):
+    """Context parallelism: rank r holds the r-th span of cp_span tokens of one sequence
+    (cp_heads query/key and value heads, D = 128, BNSD), one all-gather of the span maps.
+
+    With one process, ``--cp-emulate E`` runs the work of E ranks on this GPU one after another
+    and reports the slowest rank's time (its summary, fold and forward; the all-gather of
+    2 x heads x 64 KiB per rank is not timed), beside one forward over the whole sequence."""
+    import torch
+    import chunked_kda_prefill_b200 as kda
+
+    local = _env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    ranks = world if world > 1 else max(1, args.cp_emulate)
+    H, S_loc, D = args.cp_heads, args.cp_span, 128
+    w = W.custom(f"cp_span_1x{H}x{S_loc}", "BNSD", 1, H, H, S_loc, [S_loc], lower_bound=-5.0,
+                 init_state="zeros", seed=300 + rank)
+    inp = W.generate(w)
+    d = {n: torch.from_numpy(np.ascontiguousarray(inp[n]).view(np.int16)).view(
+        torch.bfloat16).to(dev) for n in ("q", "k", "v", "g", "beta")}
+    for n in ("A_log", "dt_bias", "initial_state"):
+        d[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).to(dev)
+    plan = kda.plan(d["q"], d["v"], d["initial_state"], "BNSD")
+    args_fwd = (d["q"], d["k"], d["v"], d["g"], d["beta"], w.scale)
+    tail = (d["A_log"], d["dt_bias"], w.lower_bound, "BNSD", plan)
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        return a.elapsed_time(b) / n
+
+    with ClockSampler(local) as clk:
+        if world > 1:
+            ms = timed(lambda: kda.flash_kda_context_parallel(*args_fwd, d["initial_state"],
+                                                              *tail), args.steps)
+            ms = _max_over_ranks(ms, dist, dev)
+            parts, whole = None, None
+        else:
+            gathered = torch.zeros((ranks, 2, 1, H, D, D), dtype=torch.float32, device=dev)
+            t_sum = timed(lambda: kda.forward_summary(
+                d["q"], d["k"], d["v"], d["g"], d["beta"], *tail, M=gathered[0, 0],
+                R=gathered[0, 1]), args.steps)
+            t_fwd = timed(lambda: kda.flash_kda(*args_fwd, d["initial_state"], *tail),
+                          args.steps)
+            t_chain = [0.0] + [timed(lambda j=j: kda.state_chain(
+                d["initial_state"], gathered[:j, 0], gathered[:j, 1]), args.steps)
+                for j in range(1, ranks)]
+            per_rank = [(t_sum if r < ranks - 1 else 0.0) + t_chain[r] + t_fwd
+                        for r in range(ranks)]
+            ms = max(per_rank)
+            parts = {"summary_ms": t_sum, "forward_ms": t_fwd, "chain_ms": t_chain,
+                     "per_rank_ms": per_rank}
+            whole = None
+            if ranks > 1:  # the whole sequence on this one GPU, for comparison
+                wf = W.custom(f"cp_whole_1x{H}x{ranks * S_loc}", "BNSD", 1, H, H,
+                              ranks * S_loc, [ranks * S_loc], init_state="zeros", seed=301)
+                fi = W.generate(wf)
+                fd = {n: torch.from_numpy(np.ascontiguousarray(fi[n]).view(np.int16)).view(
+                    torch.bfloat16).to(dev) for n in ("q", "k", "v", "g", "beta")}
+                fplan = kda.plan(fd["q"], fd["v"], d["initial_state"], "BNSD")
+                whole = {"ms": timed(lambda: kda.flash_kda(
+                    fd["q"], fd["k"], fd["v"], fd["g"], fd["beta"], w.scale, d["initial_state"],
+                    d["A_log"], d["dt_bias"], w.lower_bound, "BNSD", fplan), args.steps),
+                    "schedule": (f"segments of {fplan.segment_chunks} chunks"
+                                 if fplan.segment_chunks > 0 else "whole units")}
+    token_heads = ranks * S_loc * H
+    line = {"metric": CP_METRIC, "value": token_heads / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 inputs)",
+            "config": {"workload": f"context_parallel_1x{H}x{S_loc}_per_rank", "ranks": ranks,
+                       "emulated": world == 1 and ranks > 1, "span_tokens": S_loc, "heads": H,
+                       "D": D, "exchange": "one all_gather of [M; R] per rank (2 x 64 KiB "
+                       "per head)" + (", not timed (ranks emulated on one GPU)"
+                                      if world == 1 else "")},
+            "clocks": clk.report(), "parts": parts, "whole_sequence_one_gpu": whole}
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -508,8 +613,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)
-    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode"],
-                    help="prefill (the default, the headline) or the single-token decode step")
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode", "cp"],
+                    help="prefill (the default, the headline), the single-token decode step, "
+                         "or context parallelism (one sequence split over the ranks)")
+    ap.add_argument("--cp-span", type=int, default=8192, help="cp: tokens per rank")
+    ap.add_argument("--cp-heads", type=int, default=3, help="cp: heads (Nqk = Nv)")
+    ap.add_argument("--cp-emulate", type=int, default=1,
+                    help="cp with one process: ranks to emulate one after another")
     ap.add_argument("--decode-batch", type=int, default=256)
     ap.add_argument("--segment-chunks", type=int, default=-1,
                     help="schedule: -1 the planner's choice, 0 whole units, n > 0 segments of n "
@@ -522,6 +632,8 @@ def main():
         return run_reference(args, rank, world)
     if args.mode == "decode":
         return run_decode(args, rank, world)
+    if args.mode == "cp":
+        return run_cp(args, rank, world)
     return run_ours(args, rank, world)
 
 

@@ -232,6 +232,75 @@ def decode(q, k, v, g, beta, scale: float, state, A_log, dt_bias, lower_bound: f
     return out, state_out
 
 
+def forward_summary(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, layout: str,
+                    plan: KdaPlan, M: torch.Tensor | None = None, R: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None,
+                    stream: torch.cuda.Stream | None = None):
+    """Every unit's affine state map over its tokens, S_end = S_start M + R (kda_forward_summary).
+
+    Returns (M, R), fp32 [B, Nv, D, D] each; no outputs are written.  M and R may be given (for
+    example two halves of one exchange buffer).
+    """
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("forward_summary runs on a CUDA device only")
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta")):
+        _expect(t, name, torch.bfloat16, dev)
+    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias")):
+        _expect(t, name, torch.float32, dev)
+    if plan.layout != layout:
+        raise KdaError(8, "plan was built for another layout")
+    sh = plan.shape
+    if M is None:
+        M = torch.empty((sh.B, sh.Nv, sh.D, sh.D), dtype=torch.float32, device=dev)
+    if R is None:
+        R = torch.empty((sh.B, sh.Nv, sh.D, sh.D), dtype=torch.float32, device=dev)
+    _expect(M, "M", torch.float32, dev)
+    _expect(R, "R", torch.float32, dev)
+    if workspace is None:
+        workspace = plan.workspace()
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    code = _lib.load().kda_forward_summary(
+        ctypes.byref(sh), plan.host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+        plan.dev.data_ptr(), plan.host.size, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+        g.data_ptr(), beta.data_ptr(), A_log.data_ptr(), dt_bias.data_ptr(), float(lower_bound),
+        workspace.data_ptr(), workspace.numel(), M.data_ptr(), R.data_ptr(), s.cuda_stream)
+    check(code, "kda_forward_summary")
+    return M, R
+
+
+def state_chain(S_in: torch.Tensor | None, M: torch.Tensor, R: torch.Tensor,
+                S_out: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """S = S_in; for j: S = S M[j] + R[j]; returns S (kda_state_chain, fp32).
+
+    M and R: [n, B, Nv, D, D] views whose per-step blocks are contiguous and equally spaced (a
+    packed stack, or the two halves of an all-gathered [world, 2, B, Nv, D, D] buffer).  S_in:
+    [B, Nv, D, D] or None (zeros).  n may be 0.
+    """
+    if M.dim() != 5 or M.shape != R.shape or M.stride() != R.stride():
+        raise ValueError("M and R must be [n, B, Nv, D, D] views with the same layout")
+    n, B, Nv, D, _ = M.shape
+    mat = B * Nv * D * D
+    if n > 0 and not (M[0].is_contiguous() and R[0].is_contiguous()):
+        raise ValueError("every step's maps must be contiguous")
+    step = M.stride(0) if n > 1 else mat
+    dev = M.device
+    for t, name in ((M, "M"), (R, "R")):
+        if t.dtype != torch.float32 or t.device != dev:
+            raise TypeError(f"{name} must be fp32 on {dev}")
+    if S_in is not None:
+        _expect(S_in, "S_in", torch.float32, dev)
+    if S_out is None:
+        S_out = torch.empty((B, Nv, D, D), dtype=torch.float32, device=dev)
+    _expect(S_out, "S_out", torch.float32, dev)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    code = _lib.load().kda_state_chain(B * Nv, D, n, _ptr(S_in), M.data_ptr() if n else None,
+                                       R.data_ptr() if n else None, int(step),
+                                       S_out.data_ptr(), s.cuda_stream)
+    check(code, "kda_state_chain")
+    return S_out
+
+
 def device_status(workspace: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
     """Synchronise and raise if the last forward on this workspace recorded a device error."""
     s = stream if stream is not None else torch.cuda.current_stream(workspace.device)

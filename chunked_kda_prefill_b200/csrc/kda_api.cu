@@ -48,11 +48,12 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
                           const float* initial_state, const float* A_log, const float* dt_bias,
                           float lower_bound, void* workspace, size_t workspace_bytes, void* out,
                           float* final_state, cudaStream_t stream, float* dbg,
-                          unsigned long long* tprof) {
+                          unsigned long long* tprof, float* sum_m) {
   kda_status_t st = validate_shape(shape);
   if (st != KDA_OK) return st;
+  const bool summary = (path == PATH_SUMMARY);  // final_state receives R, sum_m M; no out
   if (!plan_host || !plan_dev || !q || !k || !v || !g || !beta || !A_log || !dt_bias ||
-      !workspace || !out || !final_state)
+      !workspace || (!out && !summary) || !final_state || (summary && !sum_m))
     return KDA_ERR_NULL;
   st = validate_plan(plan_host, n_int32, shape);
   if (st != KDA_OK) return st;
@@ -60,7 +61,8 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   if (!std::isfinite(scale)) return KDA_ERR_LOWER_BOUND;
   if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_LOWER_BOUND;
   {
-    const void* a16[] = {q, k, v, g, out, final_state, A_log, dt_bias, plan_dev, initial_state};
+    const void* a16[] = {q, k, v, g, out, final_state, A_log, dt_bias, plan_dev, initial_state,
+                         sum_m};
     for (const void* ptr : a16)
       if (reinterpret_cast<uintptr_t>(ptr) & 15u) return KDA_ERR_ALIGN;
     if (reinterpret_cast<uintptr_t>(beta) & 1u) return KDA_ERR_ALIGN;
@@ -78,16 +80,18 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   const size_t vg_bytes = (size_t)rows * shape->Nv * D * 2;
   const size_t beta_bytes = (size_t)rows * shape->Nv * 2;
   const size_t st_bytes = (size_t)shape->B * shape->Nv * D * D * 4;
-  const Range r_out = range_of(out, vg_bytes), r_fs = range_of(final_state, st_bytes);
+  const Range r_out = summary ? Range{0, 0} : range_of(out, vg_bytes);
+  const Range r_fs = range_of(final_state, st_bytes);
+  const Range r_m = summary ? range_of(sum_m, st_bytes) : Range{0, 0};
   const Range ins[] = {range_of(q, qk_bytes), range_of(k, qk_bytes), range_of(v, vg_bytes),
                        range_of(g, vg_bytes), range_of(beta, beta_bytes),
                        range_of(workspace, need), range_of(plan_dev, n_int32 * 4),
                        initial_state ? range_of(initial_state, st_bytes) : Range{0, 0}};
   for (const Range& r : ins) {
     if (r.hi == 0) continue;
-    if (overlaps(r, r_out) || overlaps(r, r_fs)) return KDA_ERR_ALIAS;
+    if (overlaps(r, r_out) || overlaps(r, r_fs) || overlaps(r, r_m)) return KDA_ERR_ALIAS;
   }
-  if (overlaps(r_out, r_fs)) return KDA_ERR_ALIAS;
+  if (overlaps(r_out, r_fs) || overlaps(r_m, r_fs)) return KDA_ERR_ALIAS;
 
   st = check_device();
   if (st != KDA_OK) return st;
@@ -125,6 +129,19 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   cudaError_t e;
   if (path == PATH_SIMT) {
     e = launch_simt(p, plan_host[PH_TOTAL_CHUNKS], stream);
+  } else if (summary) {
+    // every unit (or, under a segmented plan, every segment) twice: from S = 0 (R) and from
+    // S = I with v = 0 (M); segment maps are then composed into the unit's
+    const long long items =
+        2LL * (p.seg_chunks > 0 ? seg_counts(plan_host).slots + p.n_units : p.n_units);
+    if (items > INT_MAX) return KDA_ERR_SHAPE;
+    p.mode = 3;
+    p.n_items = (int)items;
+    p.S0 = nullptr;
+    p.sum_m = sum_m;
+    p.sum_r = final_state;
+    e = launch_fused(p, dbg, stream);
+    if (e == cudaSuccess && p.seg_chunks > 0) e = launch_summary_combine(p, stream);
   } else if (p.seg_chunks <= 0) {
     p.mode = 0;
     p.n_items = p.n_units;
@@ -160,6 +177,48 @@ extern "C" kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* pla
   return forward_impl(PATH_FUSED, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
                       initial_state, A_log, dt_bias, lower_bound, workspace, workspace_bytes, out,
                       final_state, reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+extern "C" kda_status_t kda_forward_summary(const kda_shape_t* shape, const int32_t* plan_host,
+                                            const int32_t* plan_dev, size_t n_int32,
+                                            const void* q, const void* k, const void* v,
+                                            const void* g, const void* beta, const float* A_log,
+                                            const float* dt_bias, float lower_bound,
+                                            void* workspace, size_t workspace_bytes,
+                                            float* M_out, float* R_out, kda_stream_t stream) {
+  // scale only weights the outputs, which a summary does not write
+  return forward_impl(PATH_SUMMARY, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, 1.0f,
+                      nullptr, A_log, dt_bias, lower_bound, workspace, workspace_bytes, nullptr,
+                      R_out, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, M_out);
+}
+
+extern "C" kda_status_t kda_state_chain(int32_t units, int32_t D, int32_t n_steps,
+                                        const float* S_in, const float* M, const float* R,
+                                        int64_t step_stride, float* S_out, kda_stream_t stream) {
+  if (D != kD && D != 64) return KDA_ERR_DIM;
+  if (units < 1 || n_steps < 0 || (long long)units > INT_MAX / 2) return KDA_ERR_SHAPE;
+  const long long mat_floats = (long long)units * D * D;
+  if (step_stride == 0) step_stride = mat_floats;
+  if (step_stride < mat_floats || (step_stride & 3)) return KDA_ERR_SHAPE;
+  if (!S_out || (n_steps > 0 && (!M || !R))) return KDA_ERR_NULL;
+  const void* a16[] = {S_in, M, R, S_out};
+  for (const void* ptr : a16)
+    if (reinterpret_cast<uintptr_t>(ptr) & 15u) return KDA_ERR_ALIGN;
+  const size_t st_bytes = (size_t)units * D * D * 4;
+  const size_t maps_bytes =
+      n_steps > 0 ? ((size_t)(n_steps - 1) * (size_t)step_stride) * 4 + st_bytes : 0;
+  const Range r_out = range_of(S_out, st_bytes);
+  // S_out may be S_in itself (each CTA reads its rows before it writes them), no other overlap
+  if (S_in && S_in != S_out && overlaps(range_of(S_in, st_bytes), r_out)) return KDA_ERR_ALIAS;
+  if (n_steps > 0 && (overlaps(range_of(M, maps_bytes), r_out) ||
+                      overlaps(range_of(R, maps_bytes), r_out)))
+    return KDA_ERR_ALIAS;
+  kda_status_t st = check_device();
+  if (st != KDA_OK) return st;
+  return launch_chain(units, D, n_steps, S_in, M, R, (size_t)step_stride, S_out,
+                      reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
 }
 
 // ---- internal entry points for the GPU tests (not part of include/kda.h) ----

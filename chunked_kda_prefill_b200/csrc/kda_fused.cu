@@ -162,6 +162,11 @@ struct Maps {
 // segment s, an R run (from S = 0) and an M run (from S = I with v = 0) that leave the segment's
 // affine map S -> S M_s + R_s in state slot s; mode 2 runs every later segment from its start
 // state (computed in between by the combine kernel), writing outputs and the final state.
+// Mode 3 (the summary of kda_forward_summary) runs every unit twice, item 2u from S = 0 (its
+// final state is R, to p.sum_r) and item 2u + 1 from S = I with v = 0 (M, to p.sum_m), writing
+// no outputs: the unit's affine map S -> S M + R over all its tokens.  Under a segmented plan
+// it runs every segment's pair instead (segments after the first into the state slots), and
+// kda_combine.cu composes them into the unit's maps.
 struct Item {
   int b, h, hq, tok0, L;  // the sequence, its first packed row and its length
   int c_begin, c_end;     // chunks of the sequence this item runs
@@ -177,16 +182,18 @@ __device__ __forceinline__ float* slot_ptr(const Params& p, int slot, int part) 
 }
 
 // Item i of this launch (every argument comes from the plan; see the Item comment).
-template <int DIM>
+template <int DIM, bool SUMMARY>
 __device__ Item item_of(const Params& p, int i) {
   const int32_t* R = p.plan + kPlanHeader;
-  int u = i;
-  if (p.mode != 0) {  // the unit whose item range holds i (item offsets increase along the plan)
+  const bool seg_summary = SUMMARY && p.seg_chunks > 0;  // mode 3 under a segmented plan
+  int u = SUMMARY ? (i >> 1) : i;
+  if ((!SUMMARY && p.mode != 0) || seg_summary) {
+    // the unit whose item range holds i (item offsets increase along the plan)
     int lo = 0, hi = p.n_units - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       const int base = R[mid * kPlanRecord + PR_SEG_BASE];
-      const int off = (p.mode == 1) ? mid + 2 * base : base;
+      const int off = seg_summary ? 2 * (mid + base) : (p.mode == 1) ? mid + 2 * base : base;
       if (off <= i) lo = mid; else hi = mid - 1;
     }
     u = lo;
@@ -204,6 +211,34 @@ __device__ Item item_of(const Params& p, int i) {
   const float* s0 = p.S0 ? p.S0 + bh : nullptr;
   it.ident = 0;
   it.zero_v = 0;
+  if (SUMMARY) {  // mode 3
+    it.s_in = nullptr;
+    it.write_out = 0;
+    it.pad = 0;
+    // whole units: item 2u + (0: R, 1: M).  Segmented plan: items 2 (u + base) + 2 s + (0, 1)
+    // for every segment s of unit u; segment 0's maps go to sum_r / sum_m, later ones to the
+    // state slots (base + s - 1), and the combine kernel composes them afterwards.
+    int sgm = 0, c0 = 0, c1 = nch;
+    if (seg_summary) {
+      const int base = rec[PR_SEG_BASE];
+      sgm = (i - 2 * (u + base)) >> 1;
+      c0 = sgm * p.seg_chunks;
+      c1 = min(nch, c0 + p.seg_chunks);
+    }
+    it.c_begin = c0;
+    it.c_end = c1;
+    const bool m_run = i & 1;
+    if (m_run) {
+      it.ident = 1;
+      it.zero_v = 1;
+    }
+    if (sgm == 0) {
+      it.s_out = (m_run ? p.sum_m : p.sum_r) + bh;
+    } else {
+      it.s_out = slot_ptr(p, rec[PR_SEG_BASE] + sgm - 1, m_run ? SLOT_M : SLOT_R);
+    }
+    return it;
+  }
   if (p.mode == 0) {
     it.c_begin = 0;
     it.c_end = nch;
@@ -252,11 +287,11 @@ __device__ Item item_of(const Params& p, int i) {
 struct LoadRec {
   int b, h, hq, tok0, c_begin, c_end;
 };
-template <int DIM>
+template <int DIM, bool SUMMARY>
 __device__ __forceinline__ LoadRec load_rec(const Params& p, int i) {
   LoadRec r{0, 0, 0, 0, 0, 0};
   if (i < p.n_items) {
-    const Item it = item_of<DIM>(p, i);
+    const Item it = item_of<DIM, SUMMARY>(p, i);
     r = LoadRec{it.b, it.h, it.hq, it.tok0, it.c_begin, it.c_end};
   }
   return r;
@@ -309,8 +344,8 @@ __device__ __forceinline__ void issue_box(const Params& p, const Maps& m, uint32
 }  // namespace
 
 // DIM: the tensors' head dim (128, or 64 with the upper channels zero-filled); every tile,
-// TMEM accumulator and MMA is 128 channels wide either way.
-template <int DIM>
+// TMEM accumulator and MMA is 128 channels wide either way.  SUMMARY: the mode-3 instance.
+template <int DIM, bool SUMMARY>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_kernel(const Params p, const __grid_constant__ Maps maps, float* dbg) {
   extern __shared__ uint8_t smem_raw[];
@@ -376,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pr.pu += G_stride;
       pr.cur = pr.next;
       pr.pc = pr.cur.c_begin;
-      pr.next = load_rec<DIM>(p, pr.pu + G_stride);
+      pr.next = load_rec<DIM, SUMMARY>(p, pr.pu + G_stride);
     }
   };
   auto issue_planned = [&](int box) {
@@ -387,9 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     prod->pu = blockIdx.x;
     prod->issued = 0;
-    prod->cur = load_rec<DIM>(p, blockIdx.x);
+    prod->cur = load_rec<DIM, SUMMARY>(p, blockIdx.x);
     prod->pc = prod->cur.c_begin;
-    prod->next = load_rec<DIM>(p, blockIdx.x + G_stride);
+    prod->next = load_rec<DIM, SUMMARY>(p, blockIdx.x + G_stride);
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.k);
     tma_prefetch_desc(&maps.v);
@@ -431,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t colhalf = (uint32_t)(j0 >> 6);
 
   for (int ii = blockIdx.x; ii < p.n_items && !aborted; ii += G_stride) {
-    const Item it = item_of<DIM>(p, ii);
+    const Item it = item_of<DIM, SUMMARY>(p, ii);
     const int b = it.b, h = it.h, tok0 = it.tok0, L = it.L, coff = it.coff;
     const float a_h = expf(p.A_log[h]);
     const float lbl2 = p.lower_bound * kLog2e;
@@ -1450,12 +1485,15 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kda_fused_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kFusedSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kFusedSmemBytes);
-    if (e != cudaSuccess) return e;
+    const void* fns[] = {(const void*)kda_fused_kernel<kD, false>,
+                         (const void*)kda_fused_kernel<64, false>,
+                         (const void*)kda_fused_kernel<kD, true>,
+                         (const void*)kda_fused_kernel<64, true>};
+    for (const void* f : fns) {
+      e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kFusedSmemBytes);
+      if (e != cudaSuccess) return e;
+    }
     e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     configured_device = dev;
@@ -1469,8 +1507,15 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   if (p.n_items < 1) return cudaSuccess;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
-  if (p.D == kD) kda_fused_kernel<kD><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
-  else kda_fused_kernel<64><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
+  const bool summary = (p.mode == 3);
+  if (p.D == kD && !summary)
+    kda_fused_kernel<kD, false><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
+  else if (!summary)
+    kda_fused_kernel<64, false><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
+  else if (p.D == kD)
+    kda_fused_kernel<kD, true><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
+  else
+    kda_fused_kernel<64, true><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
   return cudaGetLastError();
 }
 

@@ -31,8 +31,11 @@ struct Params {
   unsigned long long* tprof;  // optional: CTA 0 records clock64() at phase boundaries
   // work items of this launch: mode 0 = whole units; under a segmented plan (seg_chunks > 0)
   // mode 1 = the segment-summary pass, mode 2 = the output pass (see kda_plan_segmented)
+  // mode 3 = the per-unit affine summary (M, R) of kda_forward_summary
   int mode, seg_chunks, n_items;
   float* states;  // the segmented schedule's state slots (workspace after its header)
+  float* sum_m;   // mode 3: every unit's M and R, fp32 [B, Nv, D, D] each
+  float* sum_r;
 };
 
 // Element offset of the D-vector of (sequence b, head hx of NX heads, token t of the sequence).
@@ -71,8 +74,15 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream);
 // The segmented schedule's middle kernel: every unit's segment start states from the segment
 // summaries (S_{s+1} = S_s M_s + R_s, fp32).
 cudaError_t launch_combine(const Params& p, cudaStream_t stream);
+// kda_forward_summary under a segmented plan: composes every unit's segment maps into sum_m /
+// sum_r (which hold segment 0's).
+cudaError_t launch_summary_combine(const Params& p, cudaStream_t stream);
+// kda_state_chain's kernel: S_out[u] = fold of S <- S M_j[u] + R_j[u] from S_in[u] (null: 0);
+// step j's maps start step_stride floats after step j-1's.
+cudaError_t launch_chain(int units, int D, int n_steps, const float* S_in, const float* M,
+                         const float* R, size_t step_stride, float* S_out, cudaStream_t stream);
 
-enum ForwardPath : int { PATH_FUSED = 0, PATH_SIMT = 1 };
+enum ForwardPath : int { PATH_FUSED = 0, PATH_SIMT = 1, PATH_SUMMARY = 2 };
 
 // Shared body of the forward entry points: every host check, then the launches of `path`.
 kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* plan_host,
@@ -81,7 +91,7 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
                           const float* initial_state, const float* A_log, const float* dt_bias,
                           float lower_bound, void* workspace, size_t workspace_bytes, void* out,
                           float* final_state, cudaStream_t stream, float* dbg,
-                          unsigned long long* tprof = nullptr);
+                          unsigned long long* tprof = nullptr, float* sum_m = nullptr);
 
 // Workspace bytes of the two-kernel path for a validated plan.
 size_t simt_workspace_bytes(const int32_t* plan);

@@ -156,6 +156,51 @@ KDA_API kda_status_t kda_forward(const kda_shape_t* shape, const int32_t* plan_h
                          float lower_bound, void* workspace, size_t workspace_bytes, void* out,
                          float* final_state, kda_stream_t stream);
 
+/* The affine summary of every unit (context parallelism, step 1).  Per chunk the state update
+ * is affine in the start state (the FlashKDA README's chunk equations, 功能说明, rearranged):
+ * S_next = S M_c + R_c with M_c = Diag(gamma_C) - W^T K^ and R_c = U^T K^.  Over all the tokens
+ * a unit holds, S_end = S_start M + R; this call writes M (the final state from S = I with
+ * v = 0) and R (the final state from S = 0) of every unit, without outputs.
+ *   shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, A_log, dt_bias, lower_bound,
+ *   workspace, workspace_bytes: as for kda_forward (scale is not needed: it weights only the
+ *                  outputs).  Under a segmented plan every segment's pair of maps is computed in
+ *                  parallel (segments after a unit's first into the workspace's state slots) and
+ *                  a second kernel composes them in fp32, M = M_0 M_1 ..., R = (R_0 M_1 + R_1)
+ *                  M_2 + ...; otherwise every unit runs whole, twice.
+ *   M_out, R_out : fp32 [B,Nv,D(Dv),D(Dk)] each, caller-owned, 16-byte aligned; they must not
+ *                  overlap each other or any input (KDA_ERR_ALIAS).
+ * Errors as kda_forward.  Asynchronous on `stream`. */
+KDA_API kda_status_t kda_forward_summary(const kda_shape_t* shape, const int32_t* plan_host,
+                                         const int32_t* plan_dev, size_t n_int32, const void* q,
+                                         const void* k, const void* v, const void* g,
+                                         const void* beta, const float* A_log,
+                                         const float* dt_bias, float lower_bound,
+                                         void* workspace, size_t workspace_bytes, float* M_out,
+                                         float* R_out, kda_stream_t stream);
+
+/* Fold of affine state maps (context parallelism, step 2; the same step as the segmented
+ * schedule's middle kernel): for every unit u,
+ *     S = S_in[u];  for j = 0 .. n_steps-1:  S = S M[j][u] + R[j][u];  S_out[u] = S
+ * in fp32.  Rank r of a context-parallel group starts its span from the fold over the maps of
+ * ranks 0 .. r-1.
+ *   units        : number of D x D states (>= 1), e.g. B * Nv.
+ *   D            : 128 or 64.
+ *   n_steps      : >= 0; 0 copies S_in (or zeros) to S_out.
+ *   S_in         : fp32 [units][D][D] or NULL for zeros.
+ *   M, R         : fp32; step j's maps are [units][D][D] at M + j*step_stride and
+ *                  R + j*step_stride (may be NULL when n_steps == 0).
+ *   step_stride  : floats between consecutive steps' maps; 0 means units*D*D (maps packed
+ *                  step-major); else >= units*D*D and a multiple of 4 (KDA_ERR_SHAPE).  An
+ *                  all-gather of [M; R] pairs is read in place with M, M + units*D*D and
+ *                  step_stride = 2*units*D*D.
+ *   S_out        : fp32 [units][D][D]; may be S_in itself, must not overlap it otherwise, nor M
+ *                  or R (KDA_ERR_ALIAS).
+ * All pointers are device memory, 16-byte aligned (KDA_ERR_ALIGN).  Errors: KDA_ERR_DIM,
+ * _SHAPE, _NULL, _ALIGN, _ALIAS, _DEVICE, _CUDA.  Asynchronous on `stream`. */
+KDA_API kda_status_t kda_state_chain(int32_t units, int32_t D, int32_t n_steps,
+                                     const float* S_in, const float* M, const float* R,
+                                     int64_t step_stride, float* S_out, kda_stream_t stream);
+
 /* Synchronise `stream` and return the device-side status recorded in `workspace` by the last
  * kda_forward that used it (KDA_OK, KDA_ERR_PLAN or KDA_ERR_TIMEOUT), or KDA_ERR_CUDA. */
 KDA_API kda_status_t kda_device_status(const void* workspace, kda_stream_t stream);

@@ -174,6 +174,22 @@ def test_head_dim_64_plans(L):
         assert ws.value >= 256
 
 
+def test_state_chain_argument_checks(L):
+    c = lambda units=2, D=128, n=1, S_in=0x10000000, M=0x20000000, R=0x30000000, stride=0, \
+        S_out=0x40000000: L.kda_state_chain(units, D, n, S_in, M, R, stride, S_out, None)  # noqa: E731
+    assert c(D=96) == 5
+    assert c(units=0) == 3
+    assert c(n=-1) == 3
+    assert c(stride=100) == 3                   # below units * D * D
+    assert c(stride=2 * 128 * 128 * 2 + 1) == 3  # not a multiple of 4
+    assert c(S_out=None) == 1
+    assert c(M=None) == 1
+    assert c(n=0, M=None, R=None, S_out=None) == 1
+    assert c(M=0x20000004) == 14                # M not 16-byte aligned
+    assert c(S_in=0x40000010) == 9              # S_in overlaps S_out without being it
+    assert c(R=0x40000000 - 4 * 128 * 128) == 9  # R (2 states, 128 KiB) runs into S_out
+
+
 def test_decode_argument_checks(L):
     assert _dec(L, D=96) == 5
     assert _dec(L, D=256) == 5
