@@ -13,10 +13,11 @@
 //     T = stril(diag(beta) K~ K-^T), rows 64-127 give Aqk = tril(Q~ K-^T)
 //   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 16x16 diagonal blocks and two merge levels;
 //     Xsol = X diag(beta) -> bf16 hi and lo parts stacked as one 128-row operand
-//   4 MMA  W^T = K~^T [Xsol_hi; Xsol_lo]^T (one N=128 chain), U^T = V^T Xsol^T; S <- S Diag(2^G_last)
+//   4 MMA  W^T = K~^T [Xsol_hi; Xsol_lo]^T and U^T = V^T [Xsol_hi; Xsol_lo]^T (one N=128 chain
+//          each, hi and lo parts side by side); S <- S Diag(2^G_last)
 //     meanwhile.  Then -W -> bf16 hi and lo, stored token-major over the K~ and V tiles
 //   5 MMA  [O^T | Da | Db] = S_hi [Q~ | -W_hi | -W_lo]^T (N=192) and [O^T | Da] += S_lo [Q~ | -W_hi]^T
-//     (A operand = bf16 state in TMEM); Delta^T = U^T + Da + Db
+//     (A operand = bf16 state in TMEM), Da and Db accumulating onto U's two parts; Delta^T = Da + Db
 //   6 Delta^T -> bf16 hi and lo in TMEM
 //   7 MMA  S += Delta^T K^ (hi/lo),  O^T += Delta^T Aqk^T   (then TMA for the chunk after next)
 //   8 O^T -> bf16 out (TMA store);  S -> bf16 hi and lo state operand (fp32 final_state at the end)
@@ -60,10 +61,10 @@ constexpr uint32_t kWaitLimit = 1u << 26;
 constexpr uint32_t TC_S = 0;      // state S, fp32 [Dv lanes][Dk cols]
 constexpr uint32_t TC_D = 128;    // phases 2-3: intra D_0..D_3 (160 cols)
 constexpr uint32_t TC_W = 128;    // phase 4: W^T partial products, Xsol_hi part | Xsol_lo part
-constexpr uint32_t TC_O = 128;    // phases 5-8: O^T [Dv][64 tokens]
-constexpr uint32_t TC_DA = 192;   // phase 5: S_hi (-W_hi)^T + S_lo (-W_hi)^T
-constexpr uint32_t TC_DB = 256;   // phase 5: S_hi (-W_lo)^T
-constexpr uint32_t TC_U = 320;    // phases 4-6: U^T
+constexpr uint32_t TC_U = 256;    // phase 4: U^T partial products, Xsol_hi part | Xsol_lo part
+constexpr uint32_t TC_O = 192;    // phases 5-8: O^T [Dv][64 tokens] (zeroed after phase 4)
+constexpr uint32_t TC_DA = 256;   // phase 5: U_hi part + S_hi (-W_hi)^T + S_lo (-W_hi)^T
+constexpr uint32_t TC_DB = 320;   // phase 5: U_lo part + S_hi (-W_lo)^T;  Delta^T = DA + DB
 constexpr uint32_t TC_SHI = 384;  // bf16 state operand hi (64 cols = 128 bf16 per lane)
 constexpr uint32_t TC_SLO = 448;  // bf16 state operand lo
 constexpr uint32_t TC_DHI = 384;  // phases 6-7: bf16 Delta^T operand hi (32 cols), over TC_SHI
@@ -344,8 +345,11 @@ __device__ __forceinline__ void issue_box(const Params& p, const Maps& m, uint32
 }  // namespace
 
 // DIM: the tensors' head dim (128, or 64 with the upper channels zero-filled); every tile,
-// TMEM accumulator and MMA is 128 channels wide either way.  SUMMARY: the mode-3 instance.
-template <int DIM, bool SUMMARY>
+// TMEM accumulator and MMA is 128 channels wide either way.  KIND: KIND_FORWARD (modes 0-2),
+// KIND_SUMMARY (mode 3), or KIND_DEBUG (mode 0 that also dumps every chunk's intermediates to
+// `dbg`; a separate instance, so the dump code takes no registers from the others).
+enum : int { KIND_FORWARD = 0, KIND_SUMMARY = 1, KIND_DEBUG = 2 };
+template <int DIM, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_kernel(const Params p, const __grid_constant__ Maps maps, float* dbg) {
   extern __shared__ uint8_t smem_raw[];
@@ -411,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pr.pu += G_stride;
       pr.cur = pr.next;
       pr.pc = pr.cur.c_begin;
-      pr.next = load_rec<DIM, SUMMARY>(p, pr.pu + G_stride);
+      pr.next = load_rec<DIM, KIND == KIND_SUMMARY>(p, pr.pu + G_stride);
     }
   };
   auto issue_planned = [&](int box) {
@@ -422,9 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     prod->pu = blockIdx.x;
     prod->issued = 0;
-    prod->cur = load_rec<DIM, SUMMARY>(p, blockIdx.x);
+    prod->cur = load_rec<DIM, KIND == KIND_SUMMARY>(p, blockIdx.x);
     prod->pc = prod->cur.c_begin;
-    prod->next = load_rec<DIM, SUMMARY>(p, blockIdx.x + G_stride);
+    prod->next = load_rec<DIM, KIND == KIND_SUMMARY>(p, blockIdx.x + G_stride);
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.k);
     tma_prefetch_desc(&maps.v);
@@ -466,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t colhalf = (uint32_t)(j0 >> 6);
 
   for (int ii = blockIdx.x; ii < p.n_items && !aborted; ii += G_stride) {
-    const Item it = item_of<DIM, SUMMARY>(p, ii);
+    const Item it = item_of<DIM, KIND == KIND_SUMMARY>(p, ii);
     const int b = it.b, h = it.h, tok0 = it.tok0, L = it.L, coff = it.coff;
     const float a_h = expf(p.A_log[h]);
     const float lbl2 = p.lower_bound * kLog2e;
@@ -1158,8 +1162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) {
         tc_fence_after();
         // K~ and V are MN-major A operands (rows = tokens s, the two column halves QGV_ATOM apart)
+        // (W and U alike: B = [Xsol_hi ; Xsol_lo], one N=128 operand; the two halves of each
+        // product are summed later, W in its epilogue, U by the phase-5 accumulation)
         const uint32_t idesc_w = idesc_bf16(128, 128, 1, 0);
-        const uint32_t idesc_u = idesc_bf16(128, 64, 1, 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t aw = smem_desc(as + OFF_G + kk * 2048, QGV_ATOM, 1024);
@@ -1169,8 +1174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t av = smem_desc(as + OFF_V + kk * 2048, QGV_ATOM, 1024);
-          mma_ss(tbase + TC_U, av, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc_u, kk > 0);
-          mma_ss(tbase + TC_U, av, smem_desc(sbase + SM_XSOL + 8192 + kk * 32, 16, 1024), idesc_u, 1);
+          mma_ss(tbase + TC_U, av, smem_desc(sbase + SM_XSOL + kk * 32, 16, 1024), idesc_w, kk > 0);
         }
         mma_commit(bar_mma_u);  // the U MMAs are waited for only before -W lo overwrites V
       }
@@ -1237,19 +1241,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint32_t*>(sq + OFF_V + atom_off(QGV_ATOM, r, j & ~1)) = wlo[q];
         }
       }
-      if (dbg && !it.zero_v) {  // per-chunk intermediates in the two-kernel workspace layout (fp32)
+      if (KIND == KIND_DEBUG && dbg && !it.zero_v) {
+        // per-chunk intermediates in the two-kernel workspace layout (fp32)
         float* dc = dbg + (size_t)(coff + c) * (kWsChunkBytes / 4);
         const int i = wq + lane;
         if (wg == 0) {
           for (int ch = 0; ch < 4; ++ch) {
-            uint32_t wa[16], wb[16], v[16];
+            uint32_t wa[16], wb[16], ua[16], ub[16];
             tmem_ld16(tl + TC_W + 16 * ch, wa);
             tmem_ld16(tl + TC_W + 64 + 16 * ch, wb);
-            tmem_ld16(tl + TC_U + 16 * ch, v);
+            tmem_ld16(tl + TC_U + 16 * ch, ua);
+            tmem_ld16(tl + TC_U + 64 + 16 * ch, ub);
             tmem_wait_ld();
             for (int e = 0; e < 16; ++e) {
               dc[kWsW / 4 + (16 * ch + e) * kD + i] = __uint_as_float(wa[e]) + __uint_as_float(wb[e]);
-              dc[kWsU / 4 + (16 * ch + e) * kD + i] = __uint_as_float(v[e]);
+              dc[kWsU / 4 + (16 * ch + e) * kD + i] = __uint_as_float(ua[e]) + __uint_as_float(ub[e]);
             }
           }
         }
@@ -1263,6 +1269,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           dc[kWsAqk / 4 + e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + SM_AQK + sw128_offset(64, r, s)));
         }
         if (tid < kD) dc[kWsGc / 4 + tid] = gcs[tid];
+        __syncthreads();  // every read of W's lo half is done before it is zeroed below
+      }
+      {
+        // O^T accumulates from zero in phase 5 (its MMAs add to DA and DB, which hold U): clear
+        // this thread's 16 columns of it, the W lo half this thread has read
+        tmem_st16_zero(tl + TC_O + 16 * wg);
+        tmem_wait_st();
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -1278,7 +1291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bd = smem_desc(as + (kk >> 2) * QGV_ATOM + (kk & 3) * 32, 16, 1024);
-          mma_ts(tbase + TC_O, tbase + TC_SHI + kk * 8, bd, idesc_3, kk > 0);
+          mma_ts(tbase + TC_O, tbase + TC_SHI + kk * 8, bd, idesc_3, 1);
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -1298,19 +1311,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       KDA_TS(7);
       tc_fence_after();
 
-      // =================== phase 6: Delta^T = U^T + Da + Db -> bf16 hi and lo ===================
+      // =================== phase 6: Delta^T = Da + Db (U^T included) -> bf16 hi and lo ===================
       {
         // warpgroup wg converts tokens 16 wg .. 16 wg + 15
-        uint32_t va[16], vb[16], vu[16], hi[8], lo[8];
+        uint32_t va[16], vb[16], hi[8], lo[8];
         tmem_ld16(tl + TC_DA + 16 * wg, va);
         tmem_ld16(tl + TC_DB + 16 * wg, vb);
-        tmem_ld16(tl + TC_U + 16 * wg, vu);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float d0 = __uint_as_float(vu[2 * e]) + __uint_as_float(va[2 * e]) + __uint_as_float(vb[2 * e]);
-          const float d1 = __uint_as_float(vu[2 * e + 1]) + __uint_as_float(va[2 * e + 1]) +
-                           __uint_as_float(vb[2 * e + 1]);
+          const float d0 = __uint_as_float(va[2 * e]) + __uint_as_float(vb[2 * e]);
+          const float d1 = __uint_as_float(va[2 * e + 1]) + __uint_as_float(vb[2 * e + 1]);
           hi[e] = pack_bf16(d0, d1);
           lo[e] = split_lo(d0, d1, hi[e]);
         }
@@ -1485,10 +1496,12 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (configured_device != dev) {
-    const void* fns[] = {(const void*)kda_fused_kernel<kD, false>,
-                         (const void*)kda_fused_kernel<64, false>,
-                         (const void*)kda_fused_kernel<kD, true>,
-                         (const void*)kda_fused_kernel<64, true>};
+    const void* fns[] = {(const void*)kda_fused_kernel<kD, KIND_FORWARD>,
+                         (const void*)kda_fused_kernel<64, KIND_FORWARD>,
+                         (const void*)kda_fused_kernel<kD, KIND_SUMMARY>,
+                         (const void*)kda_fused_kernel<64, KIND_SUMMARY>,
+                         (const void*)kda_fused_kernel<kD, KIND_DEBUG>,
+                         (const void*)kda_fused_kernel<64, KIND_DEBUG>};
     for (const void* f : fns) {
       e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kFusedSmemBytes);
@@ -1507,15 +1520,18 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   if (p.n_items < 1) return cudaSuccess;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
-  const bool summary = (p.mode == 3);
-  if (p.D == kD && !summary)
-    kda_fused_kernel<kD, false><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
-  else if (!summary)
-    kda_fused_kernel<64, false><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
-  else if (p.D == kD)
-    kda_fused_kernel<kD, true><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
-  else
-    kda_fused_kernel<64, true><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg);
+  const int kind = (p.mode == 3) ? KIND_SUMMARY : dbg ? KIND_DEBUG : KIND_FORWARD;
+  const bool d128 = (p.D == kD);
+#define KDA_LAUNCH_FUSED(DIM_, KIND_) \
+  kda_fused_kernel<DIM_, KIND_><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg)
+  if (kind == KIND_FORWARD) {
+    if (d128) KDA_LAUNCH_FUSED(kD, KIND_FORWARD); else KDA_LAUNCH_FUSED(64, KIND_FORWARD);
+  } else if (kind == KIND_SUMMARY) {
+    if (d128) KDA_LAUNCH_FUSED(kD, KIND_SUMMARY); else KDA_LAUNCH_FUSED(64, KIND_SUMMARY);
+  } else {
+    if (d128) KDA_LAUNCH_FUSED(kD, KIND_DEBUG); else KDA_LAUNCH_FUSED(64, KIND_DEBUG);
+  }
+#undef KDA_LAUNCH_FUSED
   return cudaGetLastError();
 }
 
