@@ -357,6 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // K steps of 16 over the head dim in the MMAs that contract it (phases 2 and 5): at D = 64 the
+  // upper channels are zero and their steps are skipped
+  constexpr int kDimSteps = DIM / 16;
   const uint32_t wq = (uint32_t)(warp & 3) * 32u;  // TMEM lane quarter of this warp
   const uint32_t wlane = wq << 16;
   const int wg = warp >> 2;  // warpgroup 0..3: each covers all 128 TMEM lanes
@@ -771,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // D[:, 0:160] = Aop [B^(0); B^(1); B^(2); B^(3)]^T in one N=160 chain: D_I = cols dcol(I)..
         const uint32_t idesc = idesc_bf16(128, BT_ROWS, 0, 0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < kDimSteps; ++kk) {
           const uint64_t ad = smem_desc(sbase + SM_AOP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           const uint64_t bd =
               smem_desc(sbase + SM_BT + (kk >> 2) * (BT_ROWS * 128) + (kk & 3) * 32, 16, 1024);
@@ -1202,7 +1205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(tl + TC_S + col, v);
           tmem_st16(tl + TC_S + col + 16, w2);
         };
-        if (warp != 0) decay(wg * 32);
+        if (warp != 0 && wg * 32 < DIM) decay(wg * 32);  // (D = 64: columns past D unused)
         if (warp == 4) decay(0);
         tmem_wait_st();
       }
@@ -1289,12 +1292,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t idesc_3 = idesc_bf16(128, 192, 0, 0);
         const uint32_t idesc_2 = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < kDimSteps; ++kk) {
           const uint64_t bd = smem_desc(as + (kk >> 2) * QGV_ATOM + (kk & 3) * 32, 16, 1024);
           mma_ts(tbase + TC_O, tbase + TC_SHI + kk * 8, bd, idesc_3, 1);
         }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < kDimSteps; ++kk) {
           const uint64_t bd = smem_desc(as + (kk >> 2) * QGV_ATOM + (kk & 3) * 32, 16, 1024);
           mma_ts(tbase + TC_O, tbase + TC_SLO + kk * 8, bd, idesc_2, 1);
         }
@@ -1391,8 +1394,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         KDA_TS(18);
-        uint32_t v0[16], v1[16], hi[16], lo[16];
         const int col = wg * 32;
+        // (D = 64: state columns past D stay out of every product, phase 5 skipping their K
+        // steps, so warpgroups 2 and 3 have nothing to convert)
+        if (col < DIM) {
+        uint32_t v0[16], v1[16], hi[16], lo[16];
         tmem_ld16(tl + TC_S + col, v0);
         tmem_ld16(tl + TC_S + col + 16, v1);
         tmem_wait_ld();
@@ -1407,7 +1413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(tl + TC_SHI + col / 2, hi);
         tmem_st16(tl + TC_SLO + col / 2, lo);
-        if (last && it.s_out && i < DIM && col < DIM) {
+        if (last && it.s_out && i < DIM) {
           float* dst = it.s_out + (size_t)i * DIM + col;
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
@@ -1418,6 +1424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __uint_as_float(v1[e]), __uint_as_float(v1[e + 1]), __uint_as_float(v1[e + 2]),
                 __uint_as_float(v1[e + 3]));
           }
+        }
         }
         tmem_wait_st();
       }
