@@ -1363,8 +1363,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // =================== phase 8: out rows;  S -> bf16 operand (and final_state) ===================
       {
         const int i = wq + lane;
-        uint32_t vo[16];
+        const int col = wg * 32;
+        // O^T and (D = 128) this thread's 32 state columns in one TMEM round trip.  D = 64: state
+        // columns past D stay out of every product (phase 5 skips their K steps), so warpgroups
+        // 2 and 3 have nothing to convert and the state is loaded below, by the others only.
+        uint32_t vo[16], v0[16], v1[16];
         tmem_ld16(tl + TC_O + 16 * wg, vo);
+        if constexpr (DIM == kD) {
+          tmem_ld16(tl + TC_S + col, v0);
+          tmem_ld16(tl + TC_S + col + 16, v1);
+        }
         tmem_wait_ld();
         if (!it.write_out) {
           // a segment-summary run: only its final state is kept
@@ -1394,14 +1402,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         KDA_TS(18);
-        const int col = wg * 32;
-        // (D = 64: state columns past D stay out of every product, phase 5 skipping their K
-        // steps, so warpgroups 2 and 3 have nothing to convert)
         if (col < DIM) {
-        uint32_t v0[16], v1[16], hi[16], lo[16];
-        tmem_ld16(tl + TC_S + col, v0);
-        tmem_ld16(tl + TC_S + col + 16, v1);
-        tmem_wait_ld();
+        if constexpr (DIM != kD) {
+          tmem_ld16(tl + TC_S + col, v0);
+          tmem_ld16(tl + TC_S + col + 16, v1);
+          tmem_wait_ld();
+        }
+        uint32_t hi[16], lo[16];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float a0 = __uint_as_float(v0[2 * e]), a1 = __uint_as_float(v0[2 * e + 1]);
