@@ -798,17 +798,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* Ys = Xs + 64 * TP;                           // block products            [32][YP]
       {
         // TMEM lane quarter q4 = warp & 3 holds rows 32 (q4 & 1) .. +31 of k (q4 < 2) or q (q4 >= 2),
-        // i.e. row blocks bA = 2 (q4 & 1) and bA + 1.  The quarter's 8 items (block, 16-column
-        // chunk) are split over its 4 warps; chunks right of a block's diagonal are zero.
+        // i.e. row blocks bA = 2 (q4 & 1) and bA + 1.  Items are (block, 16-column chunk); chunks
+        // right of a block's diagonal are zero.  q rows (Aqk): the quarter's 8 items, 2 a warp.
+        // k rows (T), default solve: warps 0 and 1 take the four diagonal 16x16 blocks, all that
+        // the first solve level reads, and start it at once; warps 4, 5, 9, 13 take the six
+        // off-diagonal blocks meanwhile.
         const int q4 = warp & 3;
         const int r = (q4 & 1) * 32 + lane;
         const bool krow = q4 < 2;
         const float br = krow ? beta_s[r] : 0.f;
         const int bA = 2 * (q4 & 1);
+        auto item_at = [&](int it, int& blk, int& ch) -> bool {
+#if KDA_SOLVE_L1 == 0
+          if (krow) {
+            if (wg == 0) {  // warp 0: (0,0) (1,1); warp 1: (2,2) (3,3)
+              blk = ch = bA + it;
+              return true;
+            }
+            if (q4 == 0) {  // block row 1 has one off-diagonal chunk: warp 4
+              blk = 1;
+              ch = 0;
+              return wg == 1 && it == 0;
+            }
+            // (2,0) (2,1) | (3,0) (3,1) | (3,2) on warps 5, 9, 13
+            const int k = 2 * (wg - 1) + it;
+            blk = (k < 2) ? 2 : 3;
+            ch = (k < 2) ? k : k - 2;
+            return k < 5;
+          }
+#endif
+          const int item = 2 * wg + it;
+          blk = bA + (item >> 2);
+          ch = item & 3;
+          return true;
+        };
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
-          const int item = 2 * wg + it;
-          const int blk = bA + (item >> 2), ch = item & 3;
+          int blk, ch;
+          if (!item_at(it, blk, ch)) continue;
           const bool mine = (r >> 4) == blk;
           if (ch <= blk) {
             uint32_t v[16];
@@ -842,18 +869,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // the merges read strictly upper blocks of X that no level writes: X(0:16, 16:32) and
         // X(32:48, 48:64) (16x16), and the upper 8x8 block of each 16x16 diagonal block
-        if (tid < 128) {
-          const int blk2 = tid >> 6, rr = (tid & 63) >> 2, c4 = (tid & 3) * 4;
+        // (threads 64-255: warps 0 and 1 go on to the first level)
+        const int zt = tid - 64;
+        if (zt >= 0 && zt < 128) {
+          const int blk2 = zt >> 6, rr = (zt & 63) >> 2, c4 = (zt & 3) * 4;
           *reinterpret_cast<float4*>(Xs + (32 * blk2 + rr) * TP + 32 * blk2 + 16 + c4) =
               make_float4(0.f, 0.f, 0.f, 0.f);
-        } else if (tid < 192) {
-          const int I = (tid - 128) >> 4, rr = ((tid - 128) >> 1) & 7, c4 = (tid & 1) * 4;
+        } else if (zt >= 128 && zt < 192) {
+          const int I = (zt - 128) >> 4, rr = ((zt - 128) >> 1) & 7, c4 = (zt & 1) * 4;
           *reinterpret_cast<float4*>(Xs + (16 * I + rr) * TP + 16 * I + 8 + c4) =
               make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+#if KDA_SOLVE_L1 == 0
+      // level 1 (default) while the other warps finish the extraction: the 8x8 diagonal
+      // inverses on warps 0 and 1, then the 8->16 merges on warps 0, 1, 8 and 12 (warps 8 and 12
+      // extract nothing); barriers among those warps only
+      const bool l1_warp = warp < 2 || warp == 8 || warp == 12;
+      if (warp < 2) {
+        named_bar_sync(1, 64);  // both warps' diagonal blocks of T are in Ts
+        {
+          // level 1a: X_mm = (I + T_mm)^-1 for the eight 8x8 diagonal blocks; thread = (block,
+          // column), rows by forward substitution as dot products over the final entries
+          const int base = 8 * (tid >> 3), cc = tid & 7;
+          float x[8];
+          x[0] = (cc == 0) ? 1.f : 0.f;
+#pragma unroll
+          for (int rr = 1; rr < 8; ++rr) {
+            const float* trow = Ts + (base + rr) * TP + base;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k0 = 0; k0 < rr; k0 += 4) {
+              const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
+              const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
+            }
+            const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) Xs[(base + k) * TP + base + cc] = x[k];
+        }
+      }
+      if (l1_warp) {
+        named_bar_sync(2, 128);  // the 8x8 inverses are in Xs
+        // level 1b: X_(16I+8.., 16I..) = -X22 T21 X11 inside each 16x16 diagonal block; thread =
+        // (row rr, column cc) of blocks I0 and I0 + 1
+        const int t128 = (warp < 2 ? warp : (warp >> 2)) * 32 + lane;  // warps 0, 1, 8, 12 -> 0..127
+        const int rr = (t128 >> 3) & 7, cc = t128 & 7, I0 = 2 * (t128 >> 6);
+#pragma unroll
+        for (int I = I0; I < I0 + 2; ++I) {
+          const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
+          const float4 ta = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1);
+          const float4 tb = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1 + 4);
+          const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+          float y = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) y = fmaf(tv[k], Xs[(c1 + k) * TP + c1 + cc], y);
+          Ys[(8 * I + rr) * YP + cc] = y;
+        }
+        named_bar_sync(2, 128);
+#pragma unroll
+        for (int I = I0; I < I0 + 2; ++I) {
+          const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
+          const float4 xa = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 8);
+          const float4 xb = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 12);
+          const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+          float z = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) z = fmaf(xv[k], Ys[(8 * I + k) * YP + cc], z);
+          Xs[r1 * TP + c1 + cc] = -z;
+        }
+      }
       __syncthreads();
       KDA_TS(13);
+      KDA_TS(14);
+#else
+      __syncthreads();
+      KDA_TS(13);
+#endif
 #if KDA_SOLVE_L1 == 1
       // level 1 (variant 1): the 16x16 diagonal inverses by column forward substitution, one
       // thread per (block, column); two merge levels follow
@@ -937,60 +1033,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             z1 = fmaf(xv[k], yv.y, z1);
           }
           *reinterpret_cast<float2*>(Xs + r1 * TP + c1 + cb) = make_float2(-z0, -z1);
-        }
-      }
-      __syncthreads();
-      KDA_TS(14);
-#else
-      // level 1 (default): 8x8 inverses, then the 8->16 merges, CTA-wide
-      // level 1a: X_mm = (I + T_mm)^-1 for the eight 8x8 diagonal blocks; thread = (block, column),
-      // rows by forward substitution as dot products over the already final entries
-      if (tid < 64) {
-        const int base = 8 * (tid >> 3), cc = tid & 7;
-        float x[8];
-        x[0] = (cc == 0) ? 1.f : 0.f;
-#pragma unroll
-        for (int rr = 1; rr < 8; ++rr) {
-          const float* trow = Ts + (base + rr) * TP + base;
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int k0 = 0; k0 < rr; k0 += 4) {
-            const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
-            const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
-          }
-          const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-          x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) Xs[(base + k) * TP + base + cc] = x[k];
-      }
-      __syncthreads();
-      // level 1b: X_(16I+8.., 16I..) = -X22 T21 X11 inside each 16x16 diagonal block (8x8 merges)
-      {
-        const int I = (tid >> 6) & 3, rr = (tid >> 3) & 7, cc = tid & 7;
-        const bool act = tid < 256;
-        const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
-        if (act) {
-          const float4 ta = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1);
-          const float4 tb = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1 + 4);
-          const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-          float y = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) y = fmaf(tv[k], Xs[(c1 + k) * TP + c1 + cc], y);
-          Ys[(8 * I + rr) * YP + cc] = y;
-        }
-        __syncthreads();
-        if (act) {
-          const float4 xa = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 8);
-          const float4 xb = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 12);
-          const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-          float z = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) z = fmaf(xv[k], Ys[(8 * I + k) * YP + cc], z);
-          Xs[r1 * TP + c1 + cc] = -z;
         }
       }
       __syncthreads();

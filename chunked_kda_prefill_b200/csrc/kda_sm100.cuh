@@ -72,6 +72,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   return false;
 }
 
+// ---------------------------------------------------------------- named CTA barriers
+// bar.sync waits until `nthreads` threads (a multiple of 32) have arrived at barrier `id`
+// (1-15; 0 is __syncthreads); it orders the participants' shared-memory accesses like it.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
