@@ -832,40 +832,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           ch = item & 3;
           return true;
         };
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-          int blk, ch;
-          if (!item_at(it, blk, ch)) continue;
+        // an item's 16 columns of its block's rows -> T (fp32, scaled by beta) or Aqk (bf16),
+        // strictly lower / lower parts; chunks right of the diagonal of an Aqk block are zeroed
+        auto put = [&](int blk, int ch, const uint32_t (&v)[16]) {
           const bool mine = (r >> 4) == blk;
-          if (ch <= blk) {
-            uint32_t v[16];
-            tmem_ld16(tl + TC_D + dcol(blk) + 16 * ch, v);
-            tmem_wait_ld();
-            if (mine) {
-              if (krow) {
-#pragma unroll
-                for (int s0 = 0; s0 < 16; s0 += 4) {
-                  float f[4];
-#pragma unroll
-                  for (int e = 0; e < 4; ++e)
-                    f[e] = (16 * ch + s0 + e < r) ? br * __uint_as_float(v[s0 + e]) : 0.f;
-                  *reinterpret_cast<float4*>(Ts + r * TP + 16 * ch + s0) = make_float4(f[0], f[1], f[2], f[3]);
-                }
-              } else {
-#pragma unroll
-                for (int s0 = 0; s0 < 16; s0 += 8) {
-                  float f[8];
-#pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    f[e] = (16 * ch + s0 + e <= r) ? __uint_as_float(v[s0 + e]) : 0.f;
-                  *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch + s0)) = pack8(f);
-                }
-              }
+          if (!mine) return;
+          if (ch > blk) {
+            if (!krow) {
+              *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch)) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch + 8)) = make_uint4(0, 0, 0, 0);
             }
-          } else if (mine && !krow) {
-            *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch)) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch + 8)) = make_uint4(0, 0, 0, 0);
+          } else if (krow) {
+#pragma unroll
+            for (int s0 = 0; s0 < 16; s0 += 4) {
+              float f[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                f[e] = (16 * ch + s0 + e < r) ? br * __uint_as_float(v[s0 + e]) : 0.f;
+              *reinterpret_cast<float4*>(Ts + r * TP + 16 * ch + s0) = make_float4(f[0], f[1], f[2], f[3]);
+            }
+          } else {
+#pragma unroll
+            for (int s0 = 0; s0 < 16; s0 += 8) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                f[e] = (16 * ch + s0 + e <= r) ? __uint_as_float(v[s0 + e]) : 0.f;
+              *reinterpret_cast<uint4*>(sm + SM_AQK + sw128_offset(64, r, 16 * ch + s0)) = pack8(f);
+            }
           }
+        };
+        {
+          // both items' TMEM loads in one round trip
+          int blk0, ch0, blk1, ch1;
+          const bool has0 = item_at(0, blk0, ch0), has1 = item_at(1, blk1, ch1);
+          uint32_t va[16], vb[16];
+          // (unconditional loads: an item without data reads its block's first chunk, unused)
+          tmem_ld16(tl + TC_D + dcol(blk0) + 16 * ((has0 && ch0 <= blk0) ? ch0 : 0), va);
+          tmem_ld16(tl + TC_D + dcol(blk1) + 16 * ((has1 && ch1 <= blk1) ? ch1 : 0), vb);
+          tmem_wait_ld();
+          if (has0) put(blk0, ch0, va);
+          if (has1) put(blk1, ch1, vb);
         }
         // the merges read strictly upper blocks of X that no level writes: X(0:16, 16:32) and
         // X(32:48, 48:64) (16x16), and the upper 8x8 block of each 16x16 diagonal block
