@@ -783,6 +783,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_mma);
         plan_load();  // the chunk after next, whose boxes go out in phases 7 and 8
       }
+      if (c > it.c_begin) {
+        // the state after the previous chunk -> this chunk's bf16 hi/lo operand (phase 5), under
+        // the intra MMAs.  16 state columns at a time; warp 0 issues the MMAs, so warps 8 and
+        // 12 (its TMEM lanes) take its columns.  (D = 64: columns past D stay out of every
+        // product, phase 5 skipping their K steps.)
+        auto conv16 = [&](int c16) {
+          uint32_t v[16], hi[8], lo[8];
+          tmem_ld16(tl + TC_S + c16, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float a0 = __uint_as_float(v[2 * e]), a1 = __uint_as_float(v[2 * e + 1]);
+            hi[e] = pack_bf16(a0, a1);
+            lo[e] = split_lo(a0, a1, hi[e]);
+          }
+          tmem_st8(tl + TC_SHI + c16 / 2, hi);
+          tmem_st8(tl + TC_SLO + c16 / 2, lo);
+        };
+        if (warp != 0 && wg * 32 < DIM) {
+          conv16(wg * 32);
+          conv16(wg * 32 + 16);
+        }
+        if (warp == 8) conv16(0);
+        if (warp == 12) conv16(16);
+        tmem_wait_st();
+      }
       wait_mma();
       KDA_TS(3);
       tc_fence_after();
@@ -1413,15 +1439,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const int i = wq + lane;
         const int col = wg * 32;
-        // O^T and (D = 128) this thread's 32 state columns in one TMEM round trip.  D = 64: state
-        // columns past D stay out of every product (phase 5 skips their K steps), so warpgroups
-        // 2 and 3 have nothing to convert and the state is loaded below, by the others only.
-        uint32_t vo[16], v0[16], v1[16];
+        uint32_t vo[16];
         tmem_ld16(tl + TC_O + 16 * wg, vo);
-        if constexpr (DIM == kD) {
-          tmem_ld16(tl + TC_S + col, v0);
-          tmem_ld16(tl + TC_S + col + 16, v1);
-        }
         tmem_wait_ld();
         if (!it.write_out) {
           // a segment-summary run: only its final state is kept
@@ -1451,25 +1470,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         KDA_TS(18);
-        if (col < DIM) {
-        if constexpr (DIM != kD) {
+        // (the state's bf16 operand for the next chunk is made in that chunk's phase 2)
+        if (last && it.s_out && i < DIM && col < DIM) {
+          uint32_t v0[16], v1[16];
           tmem_ld16(tl + TC_S + col, v0);
           tmem_ld16(tl + TC_S + col + 16, v1);
           tmem_wait_ld();
-        }
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a0 = __uint_as_float(v0[2 * e]), a1 = __uint_as_float(v0[2 * e + 1]);
-          const float c0 = __uint_as_float(v1[2 * e]), c1 = __uint_as_float(v1[2 * e + 1]);
-          hi[e] = pack_bf16(a0, a1);
-          hi[8 + e] = pack_bf16(c0, c1);
-          lo[e] = split_lo(a0, a1, hi[e]);
-          lo[8 + e] = split_lo(c0, c1, hi[8 + e]);
-        }
-        tmem_st16(tl + TC_SHI + col / 2, hi);
-        tmem_st16(tl + TC_SLO + col / 2, lo);
-        if (last && it.s_out && i < DIM) {
           float* dst = it.s_out + (size_t)i * DIM + col;
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
@@ -1481,8 +1487,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __uint_as_float(v1[e + 3]));
           }
         }
-        }
-        tmem_wait_st();
       }
       fence_proxy_async_smem();
       tc_fence_before();
