@@ -646,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncthreads();
       KDA_TS(12);
-      uint2 khlo[4];  // K^ lo parts of this thread's rows, stored once the intra MMA is done
+      uint2 khlo[4];  // K^ lo parts of this thread's rows, stored under the intra MMAs
       {
         float rqv[4], rkv[4];
         uint2 qwv[4], kwv[4];  // raw q/k words, kept for the operand pass
@@ -783,6 +783,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_mma);
         plan_load();  // the chunk after next, whose boxes go out in phases 7 and 8
       }
+      // K^ lo for the phase-7 MMAs (its region's previous out tile was read by the end of phase 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint2*>(sm + SM_KLO + colhalf * 8192u + io[i]) = khlo[i];
       if (c > it.c_begin) {
         // the state after the previous chunk -> this chunk's bf16 hi/lo operand (phase 5), under
         // the intra MMAs.  16 state columns at a time; warp 0 issues the MMAs, so warps 8 and
@@ -812,9 +816,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_mma();
       KDA_TS(3);
       tc_fence_after();
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<uint2*>(sm + SM_KLO + colhalf * 8192u + io[i]) = khlo[i];
 
       // =================== phase 3: T, Aqk, solve ===================
       // fp32 scratch in the B-tile region (free once the intra MMA has completed)
