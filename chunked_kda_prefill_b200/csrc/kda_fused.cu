@@ -10,7 +10,8 @@
 //       Aop = [k^ 2^(G-ref_I) ; scale q^ 2^(G-ref_I)],  B^(I) rows = k^ 2^(ref_I - G)  (s < 16(I+1)),
 //       K~ = k^ 2^G, Q~ = scale q^ 2^G, K^ = k^ 2^(G_last - G)   (written over the raw q/k/g tiles)
 //   2 MMA  D_I = Aop B^(I)^T, I = 0..3 (M=128, N=160 for all four blocks, K=128): rows 0-63 give
-//     T = stril(diag(beta) K~ K-^T), rows 64-127 give Aqk = tril(Q~ K-^T)
+//     T = stril(diag(beta) K~ K-^T), rows 64-127 give Aqk = tril(Q~ K-^T); meanwhile K^ lo is
+//     stored and the state left by the previous chunk becomes the bf16 hi/lo state operand
 //   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 16x16 diagonal blocks and two merge levels;
 //     Xsol = X diag(beta) -> bf16 hi and lo parts stacked as one 128-row operand
 //   4 MMA  W^T = K~^T [Xsol_hi; Xsol_lo]^T and U^T = V^T [Xsol_hi; Xsol_lo]^T (one N=128 chain
@@ -20,7 +21,7 @@
 //     (A operand = bf16 state in TMEM), Da and Db accumulating onto U's two parts; Delta^T = Da + Db
 //   6 Delta^T -> bf16 hi and lo in TMEM
 //   7 MMA  S += Delta^T K^ (hi/lo),  O^T += Delta^T Aqk^T   (then TMA for the chunk after next)
-//   8 O^T -> bf16 out (TMA store);  S -> bf16 hi and lo state operand (fp32 final_state at the end)
+//   8 O^T -> bf16 out (TMA store); fp32 final_state after the item's last chunk
 // Operands that feed the state recurrence (Xsol, W, S, Delta, K^) are split into bf16 hi + lo
 // parts and multiplied as hi*hi + lo*hi + hi*lo, so the state path keeps ~16 significant bits
 // instead of bf16's 8: without that, rounding errors pile up when the gate does not decay.
