@@ -81,6 +81,25 @@ def test_long_memory_stress(lb, S, cuda_ok):
     check_full(w, W.generate(w))
 
 
+@pytest.mark.parametrize("D,lb,seg", [(128, -0.1, None), (128, 0.0, 0), (64, -0.5, None)])
+def test_max_length_single_sequence(D, lb, seg, cuda_ok):
+    """One 65,536-token sequence (the longest the FlashKDA README's constraints name), two heads:
+    the planner's default (segmented) schedule and whole units, slow or no decay, D = 128 and
+    64.  Every output row and the final state against the oracle."""
+    w = W.custom(f"maxlen_{D}_{lb}_{seg}", "BSND", 1, 1, 2, 65536, [65536], lower_bound=lb,
+                 scale=D ** -0.5, init_state="normal", seed=41, D=D)
+    inp = W.generate(w)
+    dev = to_dev(inp)
+    plan = kda.plan(dev["q"], dev["v"], dev["initial_state"], "BSND", segment_chunks=seg)
+    if seg is None:
+        assert plan.segment_chunks > 0  # 2 units of 1024 chunks: the chunk-parallel schedule
+    o_g, fs_g = run_gpu(w, inp, dev=dev, plan=plan)
+    o_r, fs_r, _ = oracle.flash_kda(inp, w.layout, w.B, w.Nqk, w.Nv, w.S, w.D, w.scale,
+                                    w.lower_bound, None)
+    compare(o_g, o_r, f"{w.name} out")
+    compare(fs_g, fs_r, f"{w.name} final_state")
+
+
 def _same(a, b):
     return np.array_equal(a.view(np.uint32) if a.dtype == np.float32 else a,
                           b.view(np.uint32) if b.dtype == np.float32 else b)
