@@ -7,6 +7,7 @@
 // [-5, 0], TND cu_seqlens a strictly increasing prefix sum from 0 to T, BNSD/BSND valid lengths
 // in [1, S]).  The Ascend-only capacity limit on Nv is not inherited.
 #include <algorithm>
+#include <cmath>
 #include <climits>
 #include <cstring>
 #include <vector>
@@ -113,15 +114,41 @@ extern "C" kda_status_t kda_plan_size(const kda_shape_t* shape, size_t* n_int32)
 
 namespace {
 
-// The segment length the default schedule picks: units run whole unless they would leave more
-// than half the SMs idle and are long enough to split; then segments are sized so that the
-// first pass (about two work items per segment) fills the SMs once.  At least 2 chunks per
-// segment: shorter segments cost more in the extra passes than they save.
-int32_t auto_segment_chunks(long long units, long long total_chunks, int32_t max_chunks,
-                            int32_t num_sms) {
-  if (units * 2 > num_sms || max_chunks < 8) return 0;
-  const long long half = std::max(1, num_sms / 2);
-  return (int32_t)std::max(2LL, (total_chunks + half - 1) / half);
+// The segment length the default schedule picks, from a cost model in units of one chunk's
+// time on one SM (measured on B200: starting a work item costs about 0.9 chunk, one step of the
+// segment start-state chain about 0.26).  With segments of n chunks, unit u has
+// nseg_u = ceil(chunks_u / n); the first pass runs sum(2 nseg_u - 1) items and the last
+// sum(nseg_u - 1), each in ceil(items / SMs) waves of n + 0.9; the chain takes
+// max(nseg_u) - 2 steps.  Whole units take one wave of the longest unit.  Splitting is only
+// considered when the units leave more than half the SMs idle (otherwise the extra passes
+// cannot pay), and the cheapest n >= 2 is taken if it beats whole units.
+int32_t auto_segment_chunks(const std::vector<int32_t>& chunks, int32_t num_sms) {
+  const long long units = (long long)chunks.size();
+  int32_t max_chunks = 0;
+  for (int32_t c : chunks) max_chunks = std::max(max_chunks, c);
+  if (units * 2 > num_sms || max_chunks < 4) return 0;
+  constexpr double kItem = 0.9, kStep = 0.26;
+  const double sms = (double)num_sms;
+  double best = (double)max_chunks + kItem;  // whole units: one wave
+  int32_t best_n = 0;
+  for (int32_t n = 2; n < max_chunks; ++n) {
+    long long items1 = 0, items3 = 0, max_seg = 0;
+    for (int32_t c : chunks) {
+      const long long nseg = (c + n - 1) / n;
+      items1 += 2 * nseg - 1;
+      items3 += nseg - 1;
+      max_seg = std::max(max_seg, nseg);
+    }
+    const double wave = (double)n + kItem;
+    const double t = std::ceil((double)items1 / sms) * wave +
+                     std::ceil((double)items3 / sms) * wave +
+                     (double)std::max(0LL, max_seg - 2) * kStep;
+    if (t < best) {
+      best = t;
+      best_n = n;
+    }
+  }
+  return best_n;
 }
 
 kda_status_t plan_impl(const kda_shape_t* shape, const int32_t* cu, int32_t num_sms,
@@ -186,9 +213,9 @@ kda_status_t plan_impl(const kda_shape_t* shape, const int32_t* cu, int32_t num_
   }
   if (total > INT_MAX) return KDA_ERR_SHAPE;
   // segment length: explicit request (> 0), none (0), or the default policy (< 0)
-  const int32_t seg = seg_request >= 0 ? seg_request
-                                       : auto_segment_chunks((long long)units.size(), total, maxc,
-                                                             num_sms);
+  std::vector<int32_t> unit_chunks(units.size());
+  for (size_t i = 0; i < units.size(); ++i) unit_chunks[i] = units[i].chunks;
+  const int32_t seg = seg_request >= 0 ? seg_request : auto_segment_chunks(unit_chunks, num_sms);
   long long seg_base = 0;
   for (size_t i = 0; i < units.size(); ++i) {
     int32_t* r = plan + kPlanHeader + i * kPlanRecord;

@@ -102,9 +102,11 @@ KDA_API kda_status_t kda_plan_size(const kda_shape_t* shape, size_t* n_int32);
  *   plan, n_int32: host output buffer and its capacity in int32 words.
  * Units are ordered longest first.  Pure host code; never touches the GPU.
  *
- * Schedule: when the units would leave more than half of num_sms idle and the longest has at
- * least 8 chunks, the plan is segmented (see kda_plan_segmented) with segments sized so that
- * about num_sms work items run at once; otherwise every unit runs whole on one CTA. */
+ * Schedule: when the units would leave more than half of num_sms idle, the plan may be
+ * segmented (see kda_plan_segmented).  The segment length is the one a cost model, counted in
+ * chunk-times on one SM, predicts fastest: waves of work items in the two passes, plus the
+ * start-state chain.  Units run whole when that is predicted faster, and always when there
+ * are more units. */
 KDA_API kda_status_t kda_plan(const kda_shape_t* shape, const int32_t* cu_seqlens_host, int32_t num_sms,
                       int32_t* plan, size_t n_int32);
 

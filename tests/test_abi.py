@@ -230,9 +230,14 @@ def _ws(L, p):
 
 
 def test_default_schedule_segments_only_few_long_units(L):
-    # 3 units of 128 chunks on 148 SMs: segmented, ~2 work items per segment fill the SMs once
+    # 3 units of 128 chunks on 148 SMs: segmented; the cost model's pick, which measured fastest
+    # (6-chunk segments: 0.296 ms against 0.323 with 3, 0.327 with 8, 1.549 whole)
     st, p = _plan(L, _shape(layout=0, B=1, Nqk=3, Nv=3, S=8192))
     assert st == 0 and p[14] == 6
+    # 32 units of 63 and 44 chunks: 11-chunk segments (0.504 ms against 0.583 with 6, 0.519
+    # with 12, 0.742 whole)
+    st, p = _plan(L, _shape(layout=1, B=2, Nqk=4, Nv=16, S=4000), cu=[0, 4000, 6777])
+    assert st == 0 and p[14] == 11
     # 128 units of 256 chunks: whole units
     st, p = _plan(L, _shape(layout=0, B=4, Nqk=32, Nv=32, S=16384))
     assert st == 0 and p[14] == 0 and _ws(L, p) == 256
