@@ -67,6 +67,51 @@ def pin_chunked_equals_recurrent_d128(seed=1, L=150, lb=-5.0, tol=1e-9):
     assert _rel(S_c, S_r) < tol, _rel(S_c, S_r)
 
 
+def pin_chunked_equals_recurrent_d64(seed=10, L=150, lb=-5.0, tol=1e-9):
+    """I1 at the second head dim the library builds (D = 64)."""
+    rng = np.random.default_rng(seed)
+    q, k, v, g, beta, S0 = _rand_unit_inputs(rng, L, 64, 64, lb)
+    o_r, S_r = oracle.recurrent(q, k, v, g, beta, 1.0 / 8.0, S0)
+    o_c, S_c = oracle.chunked(q, k, v, g, beta, 1.0 / 8.0, S0, C=64)
+    assert _rel(o_c, o_r) < tol, _rel(o_c, o_r)
+    assert _rel(S_c, S_r) < tol, _rel(S_c, S_r)
+
+
+# ---------------------------------------------------------------------------
+# I1b: a span's state map is affine in its start state.  With M the end state from S0 = I and
+# v = 0, and R the end state from S0 = 0, every S0 ends at S0 M + R; maps of consecutive spans
+# compose, and the second span run from the folded state gives the whole sequence's outputs.
+# (The identity follows from S_t = S_{t-1} Diag(e^g_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+# being affine in S_{t-1}; the chunk-parallel and context-parallel schedules rest on it.)
+# ---------------------------------------------------------------------------
+
+def pin_affine_span_map(seed=11, L1=37, L2=29, Dk=12, Dv=9, lb=-0.05, tol=1e-10):
+    rng = np.random.default_rng(seed)
+    q, k, v, g, beta, S0 = _rand_unit_inputs(rng, L1 + L2, Dk, Dv, lb)
+    o_full, S_full = oracle.recurrent(q, k, v, g, beta, SCALE, S0)
+    spans = (slice(0, L1), slice(L1, L1 + L2))
+    maps = []
+    for sp in spans:
+        # M (Dk x Dk) is the end state of a Dk-row state that starts at I and takes no values
+        n = sp.stop - sp.start
+        _, M = oracle.recurrent(q[sp], k[sp], np.zeros((n, Dk)), g[sp], beta[sp], SCALE,
+                                np.eye(Dk))
+        _, R = oracle.recurrent(q[sp], k[sp], v[sp], g[sp], beta[sp], SCALE,
+                                np.zeros((Dv, Dk)))
+        maps.append((M, R))
+    S_mid = S0 @ maps[0][0] + maps[0][1]
+    _, S_mid_ref = oracle.recurrent(q[spans[0]], k[spans[0]], v[spans[0]], g[spans[0]],
+                                    beta[spans[0]], SCALE, S0)
+    assert _rel(S_mid, S_mid_ref) < tol, _rel(S_mid, S_mid_ref)
+    S_end = S_mid @ maps[1][0] + maps[1][1]
+    assert _rel(S_end, S_full) < tol, _rel(S_end, S_full)
+    o2, S2 = oracle.recurrent(q[spans[1]], k[spans[1]], v[spans[1]], g[spans[1]],
+                              beta[spans[1]], SCALE, S_mid)
+    assert _rel(o2, o_full[spans[1]]) < tol and _rel(S2, S_full) < tol
+    # slow decays (lb near 0) keep the start state in play, so the check is not vacuous
+    assert _rel(S_full, maps[0][1] @ maps[1][0] + maps[1][1]) > 1e-3
+
+
 # ---------------------------------------------------------------------------
 # I2: beta = 0 -> pure decay, closed form
 #   S_T = S0 Diag(exp(sum_t g_t)),  o_t = scale * S0 (exp(G_t) * q_t)
@@ -314,6 +359,7 @@ def pin_structure(seed=9, D=16, tol=1e-12):
 
 
 ALL_PINS = [pin_chunked_equals_recurrent, pin_chunked_equals_recurrent_d128,
+            pin_chunked_equals_recurrent_d64, pin_affine_span_map,
             pin_beta_zero_pure_decay, pin_g_zero_textbook_delta_rule, pin_basis_keys_overwrite,
             pin_repeated_key_ema, pin_brute_force_tiny, pin_unit_lower_inverse, pin_activations,
             pin_structure]
