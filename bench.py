@@ -607,7 +607,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=5,
+                    help="1-5 the five synthetic workloads (5 = the large prefill), 6 head dim "
+                         "64, 7 the large prefill at B = 1")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -120,7 +120,7 @@ SCALE128 = 1.0 / math.sqrt(128.0)
 
 
 def workload(idx: int) -> Workload:
-    """The five synthetic workloads (1-based index), and 6: the head-dim-64 workload."""
+    """The five synthetic workloads (1-based index); 6: head dim 64; 7: the large prefill at B = 1."""
     if idx == 1:
         return Workload("tiny_bnsd_1x1x256", "BNSD", 1, 1, 1, 256, 128, [256], -5.0, SCALE128,
                         "zeros", seed=1)
@@ -141,6 +141,11 @@ def workload(idx: int) -> Workload:
         # head dim 64: the largest K = 64 shape of FLA PR 656's timing table (B=8, T=4096, H=32)
         return Workload("headdim64_bnsd_8x32x4096", "BNSD", 8, 32, 32, 4096, 64, [4096] * 8,
                         -5.0, 1.0 / math.sqrt(64.0), "zeros", seed=6)
+    if idx == 7:
+        # one batch row of the large prefill: 32 units for 148 SMs, so the default schedule cuts
+        # each unit into segments (chunk-parallel scan)
+        return Workload("single_batch_bnsd_1x32x16384", "BNSD", 1, 32, 32, 16384, 128, [16384],
+                        -5.0, SCALE128, "zeros", seed=7)
     raise ValueError(idx)
 
 

@@ -33,9 +33,10 @@ def test_workload_full_parity(idx, cuda_ok):
     check_full(w, W.generate(w))
 
 
-@pytest.mark.parametrize("idx", [4, 5])
+@pytest.mark.parametrize("idx", [4, 5, 7])
 def test_workload_sampled_parity(idx, cuda_ok):
-    """Full-size run (the benchmarked launch), oracle on a sample of whole units."""
+    """Full-size run (the benchmarked launch), oracle on a sample of whole units.  Workload 7
+    takes the segmented schedule by default, so this is that schedule at full size."""
     w = W.workload(idx)
     inp = W.generate(w)
     o_g, fs_g = run_gpu(w, inp)
