@@ -132,6 +132,43 @@ def _expect(t, name, dtype, device):
         raise ValueError(f"{name} must be on {device}")
 
 
+def _expect_shape(t, name, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise KdaError(3, f"{name} has shape {tuple(t.shape)}, the plan needs {tuple(shape)}")
+
+
+def _io_shapes(sh: KdaShape, layout: str) -> dict:
+    """Shapes the plan's problem gives every tensor (include/kda.h, tensor layouts)."""
+    B, Nqk, Nv, S, D = sh.B, sh.Nqk, sh.Nv, sh.S, sh.D
+    if layout == "BNSD":
+        qk, vg, bt = (B, Nqk, S, D), (B, Nv, S, D), (B, Nv, S)
+    elif layout == "BSND":
+        qk, vg, bt = (B, S, Nqk, D), (B, S, Nv, D), (B, S, Nv)
+    else:
+        qk, vg, bt = (S, Nqk, D), (S, Nv, D), (S, Nv)
+    return {"q": qk, "k": qk, "v": vg, "g": vg, "beta": bt, "out": vg, "A_log": (Nv,),
+            "dt_bias": (Nv, D), "state": (B, Nv, D, D)}
+
+
+def _check_inputs(plan: KdaPlan, layout: str, dev, tensors: dict) -> dict:
+    """Dtype, contiguity, device and shape of every tensor against the plan (None = absent).
+
+    The library sees only pointers, so a tensor smaller than the plan's problem must be caught
+    here, before a kernel reads past its end.
+    """
+    if plan.layout != layout:
+        raise KdaError(8, "plan was built for another layout")
+    want = _io_shapes(plan.shape, layout)
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        key = "state" if name in ("initial_state", "final_state", "M", "R") else name
+        dtype = torch.bfloat16 if key in ("q", "k", "v", "g", "beta", "out") else torch.float32
+        _expect(t, name, dtype, dev)
+        _expect_shape(t, name, want[key])
+    return want
+
+
 def flash_kda(q, k, v, g, beta, scale: float, initial_state, A_log, dt_bias, lower_bound: float,
               layout: str, plan: KdaPlan, out: torch.Tensor | None = None,
               final_state: torch.Tensor | None = None,
@@ -140,14 +177,10 @@ def flash_kda(q, k, v, g, beta, scale: float, initial_state, A_log, dt_bias, low
     dev = q.device
     if dev.type != "cuda":
         raise ValueError("flash_kda runs on a CUDA device only")
-    for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta")):
-        _expect(t, name, torch.bfloat16, dev)
-    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias")):
-        _expect(t, name, torch.float32, dev)
-    if initial_state is not None:
-        _expect(initial_state, "initial_state", torch.float32, dev)
-    if plan.layout != layout:
-        raise KdaError(8, "plan was built for another layout")
+    _check_inputs(plan, layout, dev, {"q": q, "k": k, "v": v, "g": g, "beta": beta,
+                                      "A_log": A_log, "dt_bias": dt_bias,
+                                      "initial_state": initial_state, "out": out,
+                                      "final_state": final_state})
     sh = plan.shape
     if out is None:
         out = torch.empty_like(v)
@@ -176,14 +209,12 @@ def flash_kda_noalloc(q, k, v, g, beta, scale: float, initial_state, A_log, dt_b
     final_state.  Raises KdaError(KDA_ERR_CAPACITY) for problems larger than the scratch.
     """
     dev = q.device
-    for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (out, "out")):
-        _expect(t, name, torch.bfloat16, dev)
-    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias"), (final_state, "final_state")):
-        _expect(t, name, torch.float32, dev)
-    if initial_state is not None:
-        _expect(initial_state, "initial_state", torch.float32, dev)
-    if plan.layout != layout:
-        raise KdaError(8, "plan was built for another layout")
+    if out is None or final_state is None:
+        raise ValueError("flash_kda_noalloc needs out and final_state")
+    _check_inputs(plan, layout, dev, {"q": q, "k": k, "v": v, "g": g, "beta": beta,
+                                      "A_log": A_log, "dt_bias": dt_bias,
+                                      "initial_state": initial_state, "out": out,
+                                      "final_state": final_state})
     s = stream if stream is not None else torch.cuda.current_stream(dev)
     code = _lib.load().kda_forward_noalloc(
         ctypes.byref(plan.shape), plan.host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
@@ -223,6 +254,12 @@ def decode(q, k, v, g, beta, scale: float, state, A_log, dt_bias, lower_bound: f
         state_out = torch.empty((B, Nv, D, D), dtype=torch.float32, device=dev)
     _expect(out, "out", torch.bfloat16, dev)
     _expect(state_out, "state_out", torch.float32, dev)
+    for t, name, want in ((k, "k", q.shape), (v, "v", (B, Nv, D)), (g, "g", (B, Nv, D)),
+                          (out, "out", (B, Nv, D)), (A_log, "A_log", (Nv,)),
+                          (dt_bias, "dt_bias", (Nv, D)), (state, "state", (B, Nv, D, D)),
+                          (state_out, "state_out", (B, Nv, D, D))):
+        if t is not None:
+            _expect_shape(t, name, want)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
     code = _lib.load().kda_decode(B, Nqk, Nv, D, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                   g.data_ptr(), beta.data_ptr(), float(scale), _ptr(state),
@@ -244,19 +281,13 @@ def forward_summary(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, layout
     dev = q.device
     if dev.type != "cuda":
         raise ValueError("forward_summary runs on a CUDA device only")
-    for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta")):
-        _expect(t, name, torch.bfloat16, dev)
-    for t, name in ((A_log, "A_log"), (dt_bias, "dt_bias")):
-        _expect(t, name, torch.float32, dev)
-    if plan.layout != layout:
-        raise KdaError(8, "plan was built for another layout")
+    _check_inputs(plan, layout, dev, {"q": q, "k": k, "v": v, "g": g, "beta": beta,
+                                      "A_log": A_log, "dt_bias": dt_bias, "M": M, "R": R})
     sh = plan.shape
     if M is None:
         M = torch.empty((sh.B, sh.Nv, sh.D, sh.D), dtype=torch.float32, device=dev)
     if R is None:
         R = torch.empty((sh.B, sh.Nv, sh.D, sh.D), dtype=torch.float32, device=dev)
-    _expect(M, "M", torch.float32, dev)
-    _expect(R, "R", torch.float32, dev)
     if workspace is None:
         workspace = plan.workspace()
     s = stream if stream is not None else torch.cuda.current_stream(dev)
@@ -290,9 +321,11 @@ def state_chain(S_in: torch.Tensor | None, M: torch.Tensor, R: torch.Tensor,
             raise TypeError(f"{name} must be fp32 on {dev}")
     if S_in is not None:
         _expect(S_in, "S_in", torch.float32, dev)
+        _expect_shape(S_in, "S_in", (B, Nv, D, D))
     if S_out is None:
         S_out = torch.empty((B, Nv, D, D), dtype=torch.float32, device=dev)
     _expect(S_out, "S_out", torch.float32, dev)
+    _expect_shape(S_out, "S_out", (B, Nv, D, D))
     s = stream if stream is not None else torch.cuda.current_stream(dev)
     code = _lib.load().kda_state_chain(B * Nv, D, n, _ptr(S_in), M.data_ptr() if n else None,
                                        R.data_ptr() if n else None, int(step),

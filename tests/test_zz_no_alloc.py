@@ -45,9 +45,11 @@ def test_noalloc_rejects_problems_beyond_its_scratch(cuda_ok):
     shape = kda.KdaShape(1, w.B, w.Nqk, w.Nv, w.S, w.D)
     plan = kda.make_plan(shape, w.layout, w.cu_seqlens, device="cuda")
     assert 256 + plan.total_chunks * 148480 > (64 << 20)
-    x = torch.zeros(1, dtype=torch.bfloat16, device="cuda")
-    f = torch.zeros(1, dtype=torch.float32, device="cuda")
+    sh = W.shapes(w)
+    z = lambda shape, dt=torch.bfloat16: torch.zeros(shape, dtype=dt, device="cuda")  # noqa: E731
     with pytest.raises(kda.KdaError) as e:
-        kda.flash_kda_noalloc(x, x, x, x, x, w.scale, None, f, f, w.lower_bound, w.layout, plan,
-                              x.clone(), f.clone())
+        kda.flash_kda_noalloc(z(sh["q"]), z(sh["q"]), z(sh["v"]), z(sh["v"]), z(sh["beta"]),
+                              w.scale, None, z((w.Nv,), torch.float32),
+                              z((w.Nv, w.D), torch.float32), w.lower_bound, w.layout, plan,
+                              z(sh["v"]), z((w.B, w.Nv, w.D, w.D), torch.float32))
     assert e.value.name == "KDA_ERR_CAPACITY"
