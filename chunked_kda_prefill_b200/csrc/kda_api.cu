@@ -7,6 +7,7 @@
 
 #include "kda_internal.h"
 #include "kda_layout.cuh"
+#include "kda_once.h"
 
 namespace kda {
 namespace {
@@ -22,18 +23,18 @@ Range range_of(const void* p, size_t bytes) {
   return {lo, lo + bytes};
 }
 
-// Checks that the current device is an sm_100 part; cached per device ordinal.
+// Checks that the current device is an sm_100 part; the compute capability is cached per device
+// ordinal.
 kda_status_t check_device() {
-  static int checked[64] = {0};  // 0 unknown, 1 ok, 2 bad
+  static PerDevice major_of;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
-  if (dev >= 0 && dev < 64 && checked[dev]) return checked[dev] == 1 ? KDA_OK : KDA_ERR_DEVICE;
   int major = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+  if (once_per_device(major_of, dev, &major, [](int d, int* m) {
+        return cudaDeviceGetAttribute(m, cudaDevAttrComputeCapabilityMajor, d);
+      }) != cudaSuccess)
     return KDA_ERR_CUDA;
-  const bool ok = (major == 10);
-  if (dev >= 0 && dev < 64) checked[dev] = ok ? 1 : 2;
-  return ok ? KDA_OK : KDA_ERR_DEVICE;
+  return major == 10 ? KDA_OK : KDA_ERR_DEVICE;
 }
 
 }  // namespace

@@ -18,6 +18,7 @@
 
 #include "kda_internal.h"
 #include "kda_layout.cuh"
+#include "kda_once.h"
 
 namespace kda {
 namespace {
@@ -174,19 +175,20 @@ __global__ void __launch_bounds__(2 * D) kda_chain_kernel(const ChainParams c) {
 }  // namespace
 
 cudaError_t launch_combine(const Params& p, cudaStream_t stream) {
-  static int configured_device = -1;
+  static PerDevice setup;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kda_combine_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)combine_smem<kD>());
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)combine_smem<64>());
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  int unused = 0;
+  e = once_per_device(setup, dev, &unused, [](int, int*) {
+    const cudaError_t r = cudaFuncSetAttribute(kda_combine_kernel<kD>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)combine_smem<kD>());
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(kda_combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)combine_smem<64>());
+  });
+  if (e != cudaSuccess) return e;
   if (p.D == kD) {
     const dim3 grid((unsigned)p.n_units, kD / kRowsC);
     kda_combine_kernel<kD><<<grid, 2 * kD, combine_smem<kD>(), stream>>>(p);
@@ -198,19 +200,20 @@ cudaError_t launch_combine(const Params& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_summary_combine(const Params& p, cudaStream_t stream) {
-  static int configured_device = -1;
+  static PerDevice setup;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kda_summary_combine_kernel<kD>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)combine_smem<kD>());
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_summary_combine_kernel<64>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)combine_smem<64>());
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  int unused = 0;
+  e = once_per_device(setup, dev, &unused, [](int, int*) {
+    const cudaError_t r = cudaFuncSetAttribute(kda_summary_combine_kernel<kD>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)combine_smem<kD>());
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(kda_summary_combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)combine_smem<64>());
+  });
+  if (e != cudaSuccess) return e;
   if (p.D == kD) {
     kda_summary_combine_kernel<kD><<<dim3((unsigned)p.n_units, kD / kRowsC, 2), 2 * kD,
                                      combine_smem<kD>(), stream>>>(p);
@@ -223,19 +226,20 @@ cudaError_t launch_summary_combine(const Params& p, cudaStream_t stream) {
 
 cudaError_t launch_chain(int units, int D, int n_steps, const float* S_in, const float* M,
                          const float* R, size_t step_stride, float* S_out, cudaStream_t stream) {
-  static int configured_device = -1;
+  static PerDevice setup;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kda_chain_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)combine_smem<kD>());
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_chain_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)combine_smem<64>());
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  int unused = 0;
+  e = once_per_device(setup, dev, &unused, [](int, int*) {
+    const cudaError_t r = cudaFuncSetAttribute(kda_chain_kernel<kD>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)combine_smem<kD>());
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(kda_chain_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)combine_smem<64>());
+  });
+  if (e != cudaSuccess) return e;
   const ChainParams c{units, n_steps, step_stride, S_in, M, R, S_out};
   if (D == kD) {
     kda_chain_kernel<kD><<<dim3((unsigned)units, kD / kRowsC), 2 * kD, combine_smem<kD>(),

@@ -38,6 +38,7 @@
 
 #include "kda_internal.h"
 #include "kda_layout.cuh"
+#include "kda_once.h"
 #include "kda_sm100.cuh"
 #include "kda_tmap.h"
 
@@ -1559,12 +1560,12 @@ bool make_map(CUtensorMap* m, const void* base, int layout, int B, int NX, int S
 }  // namespace
 
 cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
-  static int configured_device = -1;
-  static int num_sms = 0;
+  static PerDevice setup;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
+  int num_sms = 0;
+  e = once_per_device(setup, dev, &num_sms, [](int d, int* sms) {
     const void* fns[] = {(const void*)kda_fused_kernel<kD, KIND_FORWARD>,
                          (const void*)kda_fused_kernel<64, KIND_FORWARD>,
                          (const void*)kda_fused_kernel<kD, KIND_SUMMARY>,
@@ -1572,14 +1573,14 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
                          (const void*)kda_fused_kernel<kD, KIND_DEBUG>,
                          (const void*)kda_fused_kernel<64, KIND_DEBUG>};
     for (const void* f : fns) {
-      e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kFusedSmemBytes);
-      if (e != cudaSuccess) return e;
+      const cudaError_t r = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)kFusedSmemBytes);
+      if (r != cudaSuccess) return r;
     }
-    e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+    return cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, d);
+  });
+  if (e != cudaSuccess) return e;
+  if (num_sms < 1) return cudaErrorInvalidValue;
   Maps m;
   if (!make_map(&m.q, p.q, p.layout, p.B, p.Nqk, p.S, p.D) ||
       !make_map(&m.k, p.k, p.layout, p.B, p.Nqk, p.S, p.D) ||

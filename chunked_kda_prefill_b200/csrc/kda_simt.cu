@@ -19,6 +19,7 @@
 
 #include "kda_internal.h"
 #include "kda_layout.cuh"
+#include "kda_once.h"
 
 namespace kda {
 
@@ -310,19 +311,20 @@ __global__ void __launch_bounds__(256) kda_scan_simt_kernel(Params p) {
 }
 
 cudaError_t launch_simt(const Params& p, int total_chunks, cudaStream_t stream) {
-  static int configured_device = -1;
+  static PerDevice setup;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(kda_chunk_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSimtChunkSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_scan_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSimtScanSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  int unused = 0;
+  e = once_per_device(setup, dev, &unused, [](int, int*) {
+    const cudaError_t r = cudaFuncSetAttribute(
+        kda_chunk_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)kSimtChunkSmemBytes);
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(kda_scan_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSimtScanSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   kda_chunk_simt_kernel<<<total_chunks, 256, kSimtChunkSmemBytes, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
