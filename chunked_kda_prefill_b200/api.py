@@ -158,6 +158,9 @@ def _check_inputs(plan: KdaPlan, layout: str, dev, tensors: dict) -> dict:
     """
     if plan.layout != layout:
         raise KdaError(8, "plan was built for another layout")
+    if plan.dev.device != dev:
+        raise ValueError(f"the plan's device copy is on {plan.dev.device}, the tensors on {dev}; "
+                         "build the plan with plan(...) or make_plan(..., device=...)")
     want = _io_shapes(plan.shape, layout)
     for name, t in tensors.items():
         if t is None:
@@ -167,6 +170,13 @@ def _check_inputs(plan: KdaPlan, layout: str, dev, tensors: dict) -> dict:
         _expect(t, name, dtype, dev)
         _expect_shape(t, name, want[key])
     return want
+
+
+def _workspace_bytes(workspace: torch.Tensor, dev) -> int:
+    """Size in bytes of a caller's workspace, after checking it is contiguous memory on ``dev``."""
+    if workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError(f"workspace must be contiguous and on {dev}")
+    return workspace.numel() * workspace.element_size()
 
 
 def flash_kda(q, k, v, g, beta, scale: float, initial_state, A_log, dt_bias, lower_bound: float,
@@ -194,7 +204,8 @@ def flash_kda(q, k, v, g, beta, scale: float, initial_state, A_log, dt_bias, low
                          plan.dev.data_ptr(), plan.host.size, q.data_ptr(), k.data_ptr(),
                          v.data_ptr(), g.data_ptr(), beta.data_ptr(), float(scale),
                          _ptr(initial_state), A_log.data_ptr(), dt_bias.data_ptr(),
-                         float(lower_bound), workspace.data_ptr(), workspace.numel(),
+                         float(lower_bound), workspace.data_ptr(),
+                         _workspace_bytes(workspace, dev),
                          out.data_ptr(), final_state.data_ptr(), s.cuda_stream)
     check(code, "kda_forward")
     return out, final_state
@@ -295,7 +306,8 @@ def forward_summary(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, layout
         ctypes.byref(sh), plan.host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
         plan.dev.data_ptr(), plan.host.size, q.data_ptr(), k.data_ptr(), v.data_ptr(),
         g.data_ptr(), beta.data_ptr(), A_log.data_ptr(), dt_bias.data_ptr(), float(lower_bound),
-        workspace.data_ptr(), workspace.numel(), M.data_ptr(), R.data_ptr(), s.cuda_stream)
+        workspace.data_ptr(), _workspace_bytes(workspace, dev), M.data_ptr(), R.data_ptr(),
+        s.cuda_stream)
     check(code, "kda_forward_summary")
     return M, R
 

@@ -312,3 +312,12 @@ def test_binding_checks_tensors_against_the_plan(layout):
     with pytest.raises(kda.KdaError) as e:
         api._check_inputs(plan, other, cpu, good)
     assert e.value.code == 8
+    # a plan whose device copy is not where the tensors are (here: a host plan, meta tensors)
+    with pytest.raises(ValueError):
+        api._check_inputs(plan, layout, torch.device("meta"), {})
+    # workspace: its size in bytes, and only contiguous memory on the tensors' device
+    assert api._workspace_bytes(torch.empty(10, dtype=torch.float32), cpu) == 40
+    with pytest.raises(ValueError):
+        api._workspace_bytes(torch.empty(4, 4)[:, 0], cpu)
+    with pytest.raises(ValueError):
+        api._workspace_bytes(torch.empty(16, device="meta"), cpu)
