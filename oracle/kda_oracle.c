@@ -48,7 +48,7 @@ static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
  * graw: [n][D], dt_bias: [D], out g: [n][D]. */
 void kda_oracle_gate(int n, int D, const double* graw, const double* dt_bias, double A_log,
                      double lower_bound, double* g) {
-  const double a = exp(A_log);
+  const double a = (kda_oracle_mutation == 17) ? exp(-A_log) : exp(A_log);
   for (int t = 0; t < n; ++t)
     for (int d = 0; d < D; ++d) {
       double x = graw[(size_t)t * D + d] + dt_bias[d];
@@ -129,7 +129,8 @@ void kda_oracle_unit_lower_inverse(int n, const double* T, double* X) {
     X[(size_t)c * n + c] = 1.0;
     for (int r = c + 1; r < n; ++r) {
       double acc = 0.0;
-      for (int s = c; s < r; ++s) acc += T[(size_t)r * n + s] * X[(size_t)s * n + c];
+      for (int s = (kda_oracle_mutation == 14) ? c + 1 : c; s < r; ++s)
+        acc += T[(size_t)r * n + s] * X[(size_t)s * n + c];
       X[(size_t)r * n + c] = -acc;
     }
   }
@@ -181,7 +182,8 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
       for (int s = 0; s < n; ++s) {
         double tk = 0.0, tq = 0.0;
         for (int j = 0; j < Dk; ++j) {
-          tk += Kt[(size_t)r * Dk + j] * Kb[(size_t)s * Dk + j];
+          tk += (kda_oracle_mutation == 11) ? Kb[(size_t)r * Dk + j] * Kt[(size_t)s * Dk + j]
+                                            : Kt[(size_t)r * Dk + j] * Kb[(size_t)s * Dk + j];
           tq += Qt[(size_t)r * Dk + j] * Kb[(size_t)s * Dk + j];
         }
         T[(size_t)r * n + s] = (s < r) ? beta[c0 + r] * tk : 0.0;
@@ -194,13 +196,15 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
       for (int i = 0; i < Dv; ++i) {
         double acc = 0.0;
         for (int s = 0; s < n; ++s)
-          acc += Ai[(size_t)r * n + s] * beta[c0 + s] * v[(size_t)(c0 + s) * Dv + i];
+          acc += Ai[(size_t)r * n + s] * (kda_oracle_mutation == 15 ? 1.0 : beta[c0 + s]) *
+                 v[(size_t)(c0 + s) * Dv + i];
         U[(size_t)r * Dv + i] = acc;
       }
       for (int j = 0; j < Dk; ++j) {
         double acc = 0.0;
         for (int s = 0; s < n; ++s)
-          acc += Ai[(size_t)r * n + s] * beta[c0 + s] * Kt[(size_t)s * Dk + j];
+          acc += Ai[(size_t)r * n + s] * beta[c0 + s] *
+                 (kda_oracle_mutation == 12 ? Kb : Kt)[(size_t)s * Dk + j];
         W[(size_t)r * Dk + j] = acc;
       }
     }
@@ -208,7 +212,10 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
     for (int r = 0; r < n; ++r)
       for (int i = 0; i < Dv; ++i) {
         double acc = 0.0;
-        for (int j = 0; j < Dk; ++j) acc += W[(size_t)r * Dk + j] * S[(size_t)i * Dk + j];
+        if (kda_oracle_mutation == 16 && Dk == Dv)
+          for (int j = 0; j < Dk; ++j) acc += W[(size_t)r * Dk + j] * S[(size_t)j * Dk + i];
+        else
+          for (int j = 0; j < Dk; ++j) acc += W[(size_t)r * Dk + j] * S[(size_t)i * Dk + j];
         Dl[(size_t)r * Dv + i] = U[(size_t)r * Dv + i] - acc;
       }
     /* O = Q~ S0^T + tril(Q~ K-^T) Delta */
@@ -222,7 +229,7 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
     /* S_next = S0 Diag(gamma_last) + Delta^T (K- Diag(gamma_last)) */
     for (int i = 0; i < Dv; ++i)
       for (int j = 0; j < Dk; ++j) {
-        const double gl = exp(G[(size_t)(n - 1) * Dk + j]);
+        const double gl = exp(G[(size_t)(kda_oracle_mutation == 13 ? 0 : n - 1) * Dk + j]);
         double acc = 0.0;
         for (int r = 0; r < n; ++r) acc += Dl[(size_t)r * Dv + i] * Kb[(size_t)r * Dk + j];
         const double carry = (kda_oracle_mutation == 6) ? S[(size_t)i * Dk + j]
