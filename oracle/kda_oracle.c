@@ -24,7 +24,7 @@
  *    intra-chunk q.k matrix keeps its diagonal (row >= col) while the k.k matrix is
  *    strictly lower (row > col) and beta-scaled.
  *
- * Readings where the pages are silent (each one is listed in the design notes):
+ * Readings where the pages are silent:
  *  - gate:  g = lower_bound * sigmoid(exp(A_log) * (g_raw + dt_bias))   [parity unpinned:
  *           the pages name the inputs and the bound, not the formula]
  *  - L2 normalise: x / sqrt(sum x^2 + 1e-6)
@@ -44,7 +44,8 @@ void kda_oracle_set_mutation(int m) { kda_oracle_mutation = m; }
 /* sigmoid(x) = 1 / (1 + e^-x) */
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
-/* Gate activation (FlashKDA parameter table: g activated by A_log, dt_bias, lower_bound).
+/* Gate activation (FlashKDA README, 参数说明: the raw gate is activated from A_log, dt_bias and
+ * lower_bound; the formula itself is the reading documented in the module header).
  * graw: [n][D], dt_bias: [D], out g: [n][D]. */
 void kda_oracle_gate(int n, int D, const double* graw, const double* dt_bias, double A_log,
                      double lower_bound, double* g) {
