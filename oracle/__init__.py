@@ -11,7 +11,7 @@ widens bf16 bit patterns to fp64, and walks the three tensor layouts of the
 FlashKDA problem statement (BNSD / BSND / packed TND with cu_seqlens) unit by
 unit, where a unit is one (sequence, value head).
 
-Readings the pages leave open (also listed in the design notes):
+Readings the pages leave open:
   * gate g = lower_bound * sigmoid(exp(A_log[h]) * (g_raw + dt_bias[h])): parity
     unpinned, since the pages name the inputs but print no formula;
   * L2 normalise with eps = 1e-6 inside the square root;
