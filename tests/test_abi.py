@@ -115,6 +115,17 @@ def test_plan_capacity_and_corruption(L):
     assert L.kda_workspace_size(p.ctypes.data_as(P_I32), p.size - 1, ctypes.byref(ws)) == 8
 
 
+def gpu_visible() -> bool:
+    """True when a CUDA device is visible.  A call with placeholder pointers that passes every
+    host check would then launch kernels on those addresses, so such calls are only made on a
+    host without a GPU (where they must stop at the device check)."""
+    try:
+        import torch
+        return bool(torch.cuda.is_available())
+    except Exception:
+        return True
+
+
 def _fwd(L, shape, plan, **over):
     """kda_forward with fake (never dereferenced) device pointers; every check is on the host."""
     a = dict(q=0x10000000, k=0x20000000, v=0x30000000, g=0x40000000, beta=0x50000000,
@@ -146,7 +157,8 @@ def test_forward_argument_checks(L):
     other = _shape(layout=0, B=1, Nqk=1, Nv=1, S=512)
     assert _fwd(L, other, p) == 8                       # plan built for another shape
     # all host checks pass: what remains needs a GPU (no device here -> CUDA/device error)
-    assert _fwd(L, sh, p) in (11, 13)
+    if not gpu_visible():
+        assert _fwd(L, sh, p) in (11, 13)
 
 
 def test_status_strings(L):
@@ -207,8 +219,9 @@ def test_decode_argument_checks(L):
     assert _dec(L, out=0x30000000 + 4096) == 9          # out overlaps state_out
     # in place (state_out == state_in) and a zero initial state are allowed: the remaining
     # checks need a GPU (none here -> CUDA/device error)
-    assert _dec(L, s1=0x20000000) in (11, 13)
-    assert _dec(L, s0=None) in (11, 13)
+    if not gpu_visible():
+        assert _dec(L, s1=0x20000000) in (11, 13)
+        assert _dec(L, s0=None) in (11, 13)
 
 
 def _plan_seg(L, shape, seg, cu=None, sms=148):
