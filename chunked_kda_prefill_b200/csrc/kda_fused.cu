@@ -56,6 +56,12 @@ constexpr int kThreads = 512;
 #ifndef KDA_SOLVE_L1
 #define KDA_SOLVE_L1 0
 #endif
+// The state operand of phase 5: a bf16 hi/lo pair (1, default) or the bf16 hi part alone (0: no
+// lo conversion and 8 fewer MMAs per chunk, at a lower precision of W S^T and Q~ S^T; a variant
+// for precision/speed experiments, built with -DKDA_STATE_LO=0).
+#ifndef KDA_STATE_LO
+#define KDA_STATE_LO 1
+#endif
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kWaitLimit = 1u << 26;
 
@@ -490,7 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         const int col0 = wg * 32 + half * 16;
-        uint32_t fv[16], hi[8], lo[8];
+        uint32_t fv[16], hi[8];
+#if KDA_STATE_LO
+        uint32_t lo[8];
+#endif
 #pragma unroll
         for (int c = 0; c < 16; c += 4) {
           float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -510,11 +519,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) {
           const float x0 = __uint_as_float(fv[2 * c]), x1 = __uint_as_float(fv[2 * c + 1]);
           hi[c] = pack_bf16(x0, x1);
+#if KDA_STATE_LO
           lo[c] = split_lo(x0, x1, hi[c]);
+#endif
         }
         tmem_st16(tl + TC_S + col0, fv);
         tmem_st8(tl + TC_SHI + col0 / 2, hi);
+#if KDA_STATE_LO
         tmem_st8(tl + TC_SLO + col0 / 2, lo);
+#endif
       }
       tmem_wait_st();
     }
@@ -795,17 +808,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 12 (its TMEM lanes) take its columns.  (D = 64: columns past D stay out of every
         // product, phase 5 skipping their K steps.)
         auto conv16 = [&](int c16) {
-          uint32_t v[16], hi[8], lo[8];
+          uint32_t v[16], hi[8];
+#if KDA_STATE_LO
+          uint32_t lo[8];
+#endif
           tmem_ld16(tl + TC_S + c16, v);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float a0 = __uint_as_float(v[2 * e]), a1 = __uint_as_float(v[2 * e + 1]);
             hi[e] = pack_bf16(a0, a1);
+#if KDA_STATE_LO
             lo[e] = split_lo(a0, a1, hi[e]);
+#endif
           }
           tmem_st8(tl + TC_SHI + c16 / 2, hi);
+#if KDA_STATE_LO
           tmem_st8(tl + TC_SLO + c16 / 2, lo);
+#endif
         };
         if (warp != 0 && wg * 32 < DIM) {
           conv16(wg * 32);
@@ -1368,17 +1388,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // B rows: Q~ (0-63), -W_hi (64-127), -W_lo (128-191): one K-major tile per column half
         const uint32_t idesc_3 = idesc_bf16(128, 192, 0, 0);
-        const uint32_t idesc_2 = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
         for (int kk = 0; kk < kDimSteps; ++kk) {
           const uint64_t bd = smem_desc(as + (kk >> 2) * QGV_ATOM + (kk & 3) * 32, 16, 1024);
           mma_ts(tbase + TC_O, tbase + TC_SHI + kk * 8, bd, idesc_3, 1);
         }
+#if KDA_STATE_LO
+        const uint32_t idesc_2 = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
         for (int kk = 0; kk < kDimSteps; ++kk) {
           const uint64_t bd = smem_desc(as + (kk >> 2) * QGV_ATOM + (kk & 3) * 32, 16, 1024);
           mma_ts(tbase + TC_O, tbase + TC_SLO + kk * 8, bd, idesc_2, 1);
         }
+#endif
         mma_commit(bar_mma);
       }
       if (c + 1 < it.c_end) {
