@@ -232,6 +232,8 @@ def _config(w: W.Workload, world: int):
     in_bytes = 5 * rows * w.Nv * w.D * 2
     c["l2"] = (f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2 (126 MB); no flush"
                if in_bytes > 126e6 else "L2 flushed between steps by a 256 MB write")
+    if os.environ.get("KDA_LIB"):  # a variant build of the library (build --define ...)
+        c["library"] = os.path.basename(os.environ["KDA_LIB"])
     return c
 
 
