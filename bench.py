@@ -101,18 +101,24 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 
 def algorithmic_bytes(w: W.Workload, with_initial_state: bool) -> int:
-    """Unique HBM bytes of one forward: q,k (per qk head), v, g, beta, out, states, params."""
-    rows = w.S if w.layout == "TND" else w.B * w.S
-    qk = 2 * rows * w.Nqk * w.D * 2
-    vg_out = 3 * rows * w.Nv * w.D * 2
-    beta = rows * w.Nv * 2
+    """Unique HBM bytes of one forward: q, k (per qk head), v, g and beta of the valid rows
+    (rows past a valid length are never read), out over every storage row (those rows are written
+    as zeros), the initial and final states, A_log and dt_bias."""
+    valid = sum(w.lengths)
+    stored = w.S if w.layout == "TND" else w.B * w.S
+    qk = 2 * valid * w.Nqk * w.D * 2
+    vg = 2 * valid * w.Nv * w.D * 2
+    beta = valid * w.Nv * 2
+    out = stored * w.Nv * w.D * 2
     states = (2 if with_initial_state else 1) * w.B * w.Nv * w.D * w.D * 4
     params = w.Nv * 4 + w.Nv * w.D * 4
-    return qk + vg_out + beta + states + params
+    return qk + vg + beta + out + states + params
 
 
 def algorithmic_flops(w: W.Workload) -> float:
-    """Dense MMA flops of the chunked method per chunk-head (C=64): 11.62 MFLOP at D=128."""
+    """Dense matrix-product flops of the chunked method: per chunk-head (C = 64) five 64x64xD
+    products (K K^T, Q K^T, W, U, Aqk Delta) and three 64xDxD ones (W S^T, Q~ S^T, Delta^T K^):
+    11.53 MFLOP at D = 128.  The triangular solve (about 0.09 MFLOP, CUDA cores) is not counted."""
     per_chunk = 5 * 2 * 64 * 64 * w.D + 3 * 2 * 64 * w.D * w.D
     chunks = sum(math.ceil(L / 64) for L in w.lengths) * w.Nv
     return float(per_chunk * chunks)
