@@ -2,7 +2,6 @@
 must be bit-exact (layouts, varlen packing, GQA, padding, chaining, determinism)."""
 import numpy as np
 import pytest
-import torch
 
 import chunked_kda_prefill_b200 as kda
 import kda_workloads as W

@@ -8,7 +8,6 @@ TND, and no decay (lower_bound = 0), where the identity run carries the whole hi
 """
 import numpy as np
 import pytest
-import torch
 
 import chunked_kda_prefill_b200 as kda
 import kda_workloads as W
