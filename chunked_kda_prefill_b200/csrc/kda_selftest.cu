@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* sB = sm + 32768;       // 32 KB
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 65536);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + 65536 + 64);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t bar_a = smem_u32(bar);
 
   if (tid == 0) {
