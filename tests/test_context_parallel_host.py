@@ -6,7 +6,8 @@ docstring).  Here the three library calls are replaced by fp64 stand-ins built o
 plain matrix recurrence; the forward as the oracle from the given start state), so what is
 checked is the schedule itself: which ranks summarise, that the last rank contributes nothing,
 the order of the gathered maps, which of them each rank folds, and that the spans' outputs and
-the last rank's state equal the oracle over the whole sequence.  World sizes 2 and 3.
+the last rank's state equal the oracle over the whole sequence.  World sizes 2, 3 and 4
+(the last with GQA groups of 2).
 """
 import os
 import socket
@@ -35,9 +36,9 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _workload(world, layout):
-    return W.custom(f"cp_{layout}_{world}", layout, 2, 1, 2, world * S_LOC, [world * S_LOC] * 2,
-                    lower_bound=-1.0, init_state="normal", seed=90 + world)
+def _workload(world, layout, Nqk=1, Nv=2):
+    return W.custom(f"cp_{layout}_{world}", layout, 2, Nqk, Nv, world * S_LOC,
+                    [world * S_LOC] * 2, lower_bound=-1.0, init_state="normal", seed=90 + world)
 
 
 def _span(inp, layout, r):
@@ -120,11 +121,11 @@ class OracleOps:
         return torch.from_numpy(out), torch.from_numpy(fs)
 
 
-def _worker(rank, world, port, layout, path):
+def _worker(rank, world, port, layout, path, Nqk, Nv):
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
                             world_size=world)
     try:
-        w = _workload(world, layout)
+        w = _workload(world, layout, Nqk, Nv)
         inp = W.generate(w)
         sp = _span(inp, layout, rank)
         t = {n: torch.from_numpy(a.view(np.int16)) for n, a in sp.items()}
@@ -141,11 +142,12 @@ def _worker(rank, world, port, layout, path):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,layout", [(2, "BNSD"), (3, "BSND")])
-def test_context_parallel_schedule_gloo(world, layout, tmp_path):
+@pytest.mark.parametrize("world,layout,Nqk,Nv", [(2, "BNSD", 1, 2), (3, "BSND", 1, 2),
+                                                 (4, "BSND", 2, 4)])
+def test_context_parallel_schedule_gloo(world, layout, Nqk, Nv, tmp_path):
     path = str(tmp_path / "cp")
-    mp.spawn(_worker, args=(world, _free_port(), layout, path), nprocs=world, join=True)
-    w = _workload(world, layout)
+    mp.spawn(_worker, args=(world, _free_port(), layout, path, Nqk, Nv), nprocs=world, join=True)
+    w = _workload(world, layout, Nqk, Nv)
     inp = W.generate(w)
     ref_out, ref_fs, _ = oracle.flash_kda(inp, layout, w.B, w.Nqk, w.Nv, w.S, w.D, w.scale,
                                           w.lower_bound, form="recurrent")
