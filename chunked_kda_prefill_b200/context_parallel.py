@@ -17,6 +17,10 @@ its start state to  S_end = S_start M_r + R_r.  Then, per (sequence, value head)
 Work per rank: one summary pass (two runs of the span, no outputs), a fold of r steps and one
 forward, against one forward over all W spans on a single GPU.  The only collective is the
 all-gather.  Every step runs in libkda.so; this module only orders the calls.
+
+Every rank makes the same calls in the same order.  If a rank fails before the exchange, the
+others leave the all-gather with the backend's error (the peer's connection closing, or the
+process group's timeout), so give the group a short timeout to bound how long they wait.
 """
 from __future__ import annotations
 
