@@ -2,6 +2,9 @@
 elementwise comparison with the fp64 oracle (atol = rtol = 5e-3, FlashKDA README 精度测试)."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -72,5 +75,10 @@ def compare(gpu: np.ndarray, ref: np.ndarray, what: str):
            "rmse": float(np.sqrt(np.mean(err ** 2))) if err.size else 0.0,
            "ref_rms": float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0,
            "n_bad": int(bad.sum()), "n": int(err.size)}
+    rep["max_err_over_bar"] = float((err / bound).max(initial=0.0))
+    log = os.environ.get("KDA_PARITY_LOG")
+    if log:  # one JSON line per comparison, e.g. to follow the margins across kernel variants
+        with open(log, "a") as f:
+            f.write(json.dumps(rep) + "\n")
     assert not bad.any(), f"{what}: {rep} first bad at {np.argwhere(bad)[:3].tolist()}"
     return rep
