@@ -50,34 +50,71 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def _bind(path: str):
+    L = ctypes.CDLL(path)
+    i, d = ctypes.c_int, ctypes.c_double
+    L.kda_oracle_gate.argtypes = [i, i, _dp, _dp, d, d, _dp]
+    L.kda_oracle_beta.argtypes = [i, _dp, _dp]
+    L.kda_oracle_l2norm.argtypes = [i, i, _dp, d, _dp]
+    L.kda_oracle_recurrent.argtypes = [i, i, i, _dp, _dp, _dp, _dp, _dp, d, _dp, _dp, _dp]
+    L.kda_oracle_chunked.argtypes = [i, i, i, i, _dp, _dp, _dp, _dp, _dp, d, _dp, _dp, _dp]
+    L.kda_oracle_unit_lower_inverse.argtypes = [i, _dp, _dp]
+    L.kda_oracle_unit.argtypes = [i, i, i, i, i, _dp, _dp, _dp, _dp, _dp, _dp, d, d, d,
+                                  _dp, _dp, _dp]
+    for f in ("kda_oracle_gate", "kda_oracle_beta", "kda_oracle_l2norm",
+              "kda_oracle_recurrent", "kda_oracle_chunked",
+              "kda_oracle_unit_lower_inverse", "kda_oracle_unit"):
+        getattr(L, f).restype = None
+    return L
+
+
 def lib():
     global _lib
     with _lock:
         if _lib is None:
             build()
-            L = ctypes.CDLL(_LIB_PATH)
-            i, d = ctypes.c_int, ctypes.c_double
-            L.kda_oracle_gate.argtypes = [i, i, _dp, _dp, d, d, _dp]
-            L.kda_oracle_beta.argtypes = [i, _dp, _dp]
-            L.kda_oracle_l2norm.argtypes = [i, i, _dp, d, _dp]
-            L.kda_oracle_recurrent.argtypes = [i, i, i, _dp, _dp, _dp, _dp, _dp, d, _dp, _dp, _dp]
-            L.kda_oracle_chunked.argtypes = [i, i, i, i, _dp, _dp, _dp, _dp, _dp, d, _dp, _dp, _dp]
-            L.kda_oracle_unit_lower_inverse.argtypes = [i, _dp, _dp]
-            L.kda_oracle_unit.argtypes = [i, i, i, i, i, _dp, _dp, _dp, _dp, _dp, _dp, d, d, d,
-                                          _dp, _dp, _dp]
-            L.kda_oracle_set_mutation.argtypes = [i]
-            for f in ("kda_oracle_gate", "kda_oracle_beta", "kda_oracle_l2norm",
-                      "kda_oracle_recurrent", "kda_oracle_chunked",
-                      "kda_oracle_unit_lower_inverse", "kda_oracle_unit",
-                      "kda_oracle_set_mutation"):
-                getattr(L, f).restype = None
-            _lib = L
+            _lib = _bind(_LIB_PATH)
     return _lib
 
 
-def set_mutation(m: int) -> None:
-    """Plant mistake number m in the oracle (0 restores the correct oracle)."""
-    lib().kda_oracle_set_mutation(int(m))
+def compile_source(text: str, path: str) -> str:
+    """Compile C source `text` (a variant of kda_oracle.c) to the shared library `path`, with
+    the flags of build().  Used by the planted-mistake tests, which patch a copy of the source."""
+    os.makedirs(os.path.dirname(path), exist_ok=True)
+    src = path + ".c"
+    with open(src, "w") as f:
+        f.write(text)
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fno-fast-math",
+                           "-ffp-contract=off", "-o", path, src, "-lm"])
+    return path
+
+
+def source() -> str:
+    """The text of kda_oracle.c."""
+    with open(_SRC) as f:
+        return f.read()
+
+
+class use_library:
+    """Context manager: route every oracle call through another compiled copy of the oracle
+    (a planted-mistake variant from compile_source) and restore the real one on exit."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        lib()
+        with _lock:
+            self._saved = _lib
+            _lib = _bind(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        with _lock:
+            _lib = self._saved
+        return False
 
 
 def _c(a: np.ndarray) -> np.ndarray:

@@ -36,11 +36,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-/* Planted-mistake switch used only by the pin tests (0 = the correct oracle). */
-int kda_oracle_mutation = 0;
-
-void kda_oracle_set_mutation(int m) { kda_oracle_mutation = m; }
-
 /* sigmoid(x) = 1 / (1 + e^-x) */
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
@@ -49,11 +44,10 @@ static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
  * graw: [n][D], dt_bias: [D], out g: [n][D]. */
 void kda_oracle_gate(int n, int D, const double* graw, const double* dt_bias, double A_log,
                      double lower_bound, double* g) {
-  const double a = (kda_oracle_mutation == 17) ? exp(-A_log) : exp(A_log);
+  const double a = exp(A_log);
   for (int t = 0; t < n; ++t)
     for (int d = 0; d < D; ++d) {
-      double x = graw[(size_t)t * D + d] + dt_bias[d];
-      if (kda_oracle_mutation == 7) x = graw[(size_t)t * D + d] - dt_bias[d];
+      const double x = graw[(size_t)t * D + d] + dt_bias[d];
       g[(size_t)t * D + d] = lower_bound * sigmoid(a * x);
     }
 }
@@ -61,7 +55,7 @@ void kda_oracle_gate(int n, int D, const double* graw, const double* dt_bias, do
 /* beta = sigmoid(logit) (FlashKDA parameter table: beta arrives as write logits). */
 void kda_oracle_beta(int n, const double* logit, double* beta) {
   for (int t = 0; t < n; ++t)
-    beta[t] = (kda_oracle_mutation == 10) ? logit[t] : sigmoid(logit[t]);
+    beta[t] = sigmoid(logit[t]);
 }
 
 /* Row-wise L2 normalise, y = x / sqrt(sum x^2 + eps) (FlashKDA: in-op q/k normalise). */
@@ -69,7 +63,7 @@ void kda_oracle_l2norm(int n, int D, const double* x, double eps, double* y) {
   for (int t = 0; t < n; ++t) {
     double ss = 0.0;
     for (int d = 0; d < D; ++d) ss += x[(size_t)t * D + d] * x[(size_t)t * D + d];
-    double inv = (kda_oracle_mutation == 9) ? 1.0 / (ss + eps) : 1.0 / sqrt(ss + eps);
+    const double inv = 1.0 / sqrt(ss + eps);
     for (int d = 0; d < D; ++d) y[(size_t)t * D + d] = x[(size_t)t * D + d] * inv;
   }
 }
@@ -85,18 +79,10 @@ void kda_oracle_recurrent(int L, int Dk, int Dv, const double* q, const double* 
     const double* kt = k + (size_t)t * Dk;
     const double* qt = q + (size_t)t * Dk;
     const double* vt = v + (size_t)t * Dv;
-    /* o_t from the state before the update: a planted index mistake. */
-    if (kda_oracle_mutation == 3)
-      for (int i = 0; i < Dv; ++i) {
-        double acc = 0.0;
-        for (int j = 0; j < Dk; ++j) acc += S[(size_t)i * Dk + j] * qt[j];
-        out[(size_t)t * Dv + i] = scale * acc;
-      }
     /* S <- S Diag(exp(g_t)) */
     for (int j = 0; j < Dk; ++j) decay[j] = exp(g[(size_t)t * Dk + j]);
-    if (kda_oracle_mutation != 1)
-      for (int i = 0; i < Dv; ++i)
-        for (int j = 0; j < Dk; ++j) S[(size_t)i * Dk + j] *= decay[j];
+    for (int i = 0; i < Dv; ++i)
+      for (int j = 0; j < Dk; ++j) S[(size_t)i * Dk + j] *= decay[j];
     /* S <- S (I - beta k k^T) + beta v k^T  ==  S + beta (v - S k) k^T */
     for (int i = 0; i < Dv; ++i) {
       double acc = 0.0;
@@ -104,20 +90,15 @@ void kda_oracle_recurrent(int L, int Dk, int Dv, const double* q, const double* 
       pred[i] = acc;
     }
     for (int i = 0; i < Dv; ++i) {
-      double r = (kda_oracle_mutation == 2) ? vt[i] + pred[i] : vt[i] - pred[i];
-      double c = beta[t] * r;
+      const double c = beta[t] * (vt[i] - pred[i]);
       for (int j = 0; j < Dk; ++j) S[(size_t)i * Dk + j] += c * kt[j];
     }
     /* o_t = scale * S_t q_t */
-    if (kda_oracle_mutation != 3)
-      for (int i = 0; i < Dv; ++i) {
-        double acc = 0.0;
-        if (kda_oracle_mutation == 4 && Dk == Dv)
-          for (int j = 0; j < Dk; ++j) acc += S[(size_t)j * Dk + i] * qt[j];
-        else
-          for (int j = 0; j < Dk; ++j) acc += S[(size_t)i * Dk + j] * qt[j];
-        out[(size_t)t * Dv + i] = scale * acc;
-      }
+    for (int i = 0; i < Dv; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < Dk; ++j) acc += S[(size_t)i * Dk + j] * qt[j];
+      out[(size_t)t * Dv + i] = scale * acc;
+    }
   }
   free(decay);
   free(pred);
@@ -130,7 +111,7 @@ void kda_oracle_unit_lower_inverse(int n, const double* T, double* X) {
     X[(size_t)c * n + c] = 1.0;
     for (int r = c + 1; r < n; ++r) {
       double acc = 0.0;
-      for (int s = (kda_oracle_mutation == 14) ? c + 1 : c; s < r; ++s)
+      for (int s = c; s < r; ++s)
         acc += T[(size_t)r * n + s] * X[(size_t)s * n + c];
       X[(size_t)r * n + c] = -acc;
     }
@@ -183,13 +164,11 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
       for (int s = 0; s < n; ++s) {
         double tk = 0.0, tq = 0.0;
         for (int j = 0; j < Dk; ++j) {
-          tk += (kda_oracle_mutation == 11) ? Kb[(size_t)r * Dk + j] * Kt[(size_t)s * Dk + j]
-                                            : Kt[(size_t)r * Dk + j] * Kb[(size_t)s * Dk + j];
+          tk += Kt[(size_t)r * Dk + j] * Kb[(size_t)s * Dk + j];
           tq += Qt[(size_t)r * Dk + j] * Kb[(size_t)s * Dk + j];
         }
         T[(size_t)r * n + s] = (s < r) ? beta[c0 + r] * tk : 0.0;
-        const int keep = (kda_oracle_mutation == 5) ? (s < r) : (s <= r);
-        Aqk[(size_t)r * n + s] = keep ? tq : 0.0;
+        Aqk[(size_t)r * n + s] = (s <= r) ? tq : 0.0;
       }
     kda_oracle_unit_lower_inverse(n, T, Ai);
     /* U = A^-1 diag(beta) V,  W = A^-1 diag(beta) K~ */
@@ -197,15 +176,13 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
       for (int i = 0; i < Dv; ++i) {
         double acc = 0.0;
         for (int s = 0; s < n; ++s)
-          acc += Ai[(size_t)r * n + s] * (kda_oracle_mutation == 15 ? 1.0 : beta[c0 + s]) *
-                 v[(size_t)(c0 + s) * Dv + i];
+          acc += Ai[(size_t)r * n + s] * beta[c0 + s] * v[(size_t)(c0 + s) * Dv + i];
         U[(size_t)r * Dv + i] = acc;
       }
       for (int j = 0; j < Dk; ++j) {
         double acc = 0.0;
         for (int s = 0; s < n; ++s)
-          acc += Ai[(size_t)r * n + s] * beta[c0 + s] *
-                 (kda_oracle_mutation == 12 ? Kb : Kt)[(size_t)s * Dk + j];
+          acc += Ai[(size_t)r * n + s] * beta[c0 + s] * Kt[(size_t)s * Dk + j];
         W[(size_t)r * Dk + j] = acc;
       }
     }
@@ -213,10 +190,7 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
     for (int r = 0; r < n; ++r)
       for (int i = 0; i < Dv; ++i) {
         double acc = 0.0;
-        if (kda_oracle_mutation == 16 && Dk == Dv)
-          for (int j = 0; j < Dk; ++j) acc += W[(size_t)r * Dk + j] * S[(size_t)j * Dk + i];
-        else
-          for (int j = 0; j < Dk; ++j) acc += W[(size_t)r * Dk + j] * S[(size_t)i * Dk + j];
+        for (int j = 0; j < Dk; ++j) acc += W[(size_t)r * Dk + j] * S[(size_t)i * Dk + j];
         Dl[(size_t)r * Dv + i] = U[(size_t)r * Dv + i] - acc;
       }
     /* O = Q~ S0^T + tril(Q~ K-^T) Delta */
@@ -230,12 +204,10 @@ void kda_oracle_chunked(int L, int Dk, int Dv, int C, const double* q, const dou
     /* S_next = S0 Diag(gamma_last) + Delta^T (K- Diag(gamma_last)) */
     for (int i = 0; i < Dv; ++i)
       for (int j = 0; j < Dk; ++j) {
-        const double gl = exp(G[(size_t)(kda_oracle_mutation == 13 ? 0 : n - 1) * Dk + j]);
+        const double gl = exp(G[(size_t)(n - 1) * Dk + j]);
         double acc = 0.0;
         for (int r = 0; r < n; ++r) acc += Dl[(size_t)r * Dv + i] * Kb[(size_t)r * Dk + j];
-        const double carry = (kda_oracle_mutation == 6) ? S[(size_t)i * Dk + j]
-                                                        : S[(size_t)i * Dk + j] * gl;
-        Sn[(size_t)i * Dk + j] = carry + acc * gl;
+        Sn[(size_t)i * Dk + j] = S[(size_t)i * Dk + j] * gl + acc * gl;
       }
     memcpy(S, Sn, sizeof(double) * (size_t)Dv * Dk);
   }
