@@ -73,6 +73,12 @@ def test_shape_checks(L, kw, code):
     (0, 2, 100, [0, 0, 50], 7),           # BNSD length 0
     (0, 2, 100, [0, 101, 150], 7),        # BNSD length > S
     (1, 2, 100, [0, 60, 160], 0),         # BSND lengths 60, 100: fine
+    (1, 2, 100, [3, 60, 160], 7),         # BSND: prefix sums start at 0
+    (1, 2, 100, [0, 60, 59], 7),          # BSND: not increasing (length -1)
+    (1, 2, 100, [0, 60, 60], 7),          # BSND: an empty sequence
+    (1, 2, 100, [0, 60, 161], 7),         # BSND: second length 101 > S
+    (1, 3, 100, [0, 100, 200, 300], 0),   # BSND: every length S, cu[B] == B*S
+    (1, 3, 100, [0, 100, 250, 300], 7),   # BSND: 150 > S although cu[B] == B*S
     (2, 2, 100, [0, 37, 100], 0),
 ])
 def test_seqlen_checks(L, layout, B, S, cu, code):
