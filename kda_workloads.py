@@ -9,13 +9,16 @@ README, "参数说明" parameter table): q/k/v/g/beta are bf16 ~ N(0, 1) in one 
 BNSD / BSND / TND layouts, A_log [Nv] and dt_bias [Nv, D] are fp32 ~ N(0, 1),
 initial_state is fp32 [B, Nv, D, D] (zeros or N(0, 0.1^2)), D = 128.
 
-Draw order per workload, from ``numpy.random.default_rng(seed)``:
-q, k, v, g, beta, A_log, dt_bias, initial_state.  bf16 values are produced by
-round-to-nearest-even from the fp32 draws.
+Draws: tensor number j of q, k, v, g, beta, A_log, dt_bias, initial_state (j = 0..7) is
+filled in row-major blocks of 2^22 elements, block i from
+``numpy.random.default_rng([seed, j, i]).standard_normal(dtype=float32)``, in parallel on the
+host threads.  bf16 values are produced by round-to-nearest-even from the fp32 draws.
 """
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -27,16 +30,67 @@ LAYOUTS = ("BNSD", "BSND", "TND")
 # bf16 helpers (storage format only)
 # ----------------------------------------------------------------------------
 
+_BLOCK = 1 << 22  # elements per block of the parallel draws and conversions
+
+
+def _threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 to bf16 (round-to-nearest-even); return the uint16 bit pattern."""
+    """Round fp32 to bf16 (round-to-nearest-even); return the uint16 bit pattern.  NaN becomes
+    the quiet NaN 0x7FC0.  Works block by block on all host threads."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32)
-    nan = np.isnan(x)
-    rounding = ((u >> 16) & 1) + np.uint32(0x7FFF)
-    out = ((u + rounding) >> 16).astype(np.uint16)
-    if nan.any():
-        out[nan] = np.uint16(0x7FC0)
-    return out
+    flat = x.reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint16)
+
+    def block(i):
+        f = flat[i:i + _BLOCK]
+        u = f.view(np.uint32)
+        r = u >> np.uint32(16)
+        r &= np.uint32(1)
+        r += np.uint32(0x7FFF)
+        r += u
+        r >>= np.uint32(16)
+        o = out[i:i + _BLOCK]
+        o[...] = r
+        nan = np.isnan(f)
+        if nan.any():
+            o[nan] = np.uint16(0x7FC0)
+
+    starts = range(0, flat.size, _BLOCK)
+    if flat.size <= _BLOCK:
+        for i in starts:
+            block(i)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(block, starts))
+    return out.reshape(x.shape)
+
+
+def normal_f32(seed: int, stream: int, shape) -> np.ndarray:
+    """fp32 draws ~ N(0, 1) of the given shape: block i of 2^22 elements (row-major order) comes
+    from numpy.random.default_rng([seed, stream, i]), so the blocks are drawn in parallel and
+    every element depends only on (seed, stream, its index)."""
+    n = int(np.prod(shape, dtype=np.int64))
+    out = np.empty(n, dtype=np.float32)
+
+    def block(j):
+        i = j * _BLOCK
+        rng = np.random.default_rng([seed, stream, j])
+        out[i:i + _BLOCK] = rng.standard_normal(size=min(_BLOCK, n - i), dtype=np.float32)
+
+    nb = (n + _BLOCK - 1) // _BLOCK
+    if nb <= 1:
+        for j in range(nb):
+            block(j)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(block, range(nb)))
+    return out.reshape(shape)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -178,20 +232,17 @@ def generate(w: Workload, pad_value: float | None = None) -> dict:
     valid length (BNSD/BSND rows >= len_b) is overwritten with it, e.g. NaN to
     prove padding is never read.
     """
-    rng = np.random.default_rng(w.seed)
     sh = shapes(w)
     out = {}
-    for name, key in (("q", "q"), ("k", "q"), ("v", "v"), ("g", "v"), ("beta", "beta")):
-        x = rng.standard_normal(size=sh[key], dtype=np.float32)
-        out[name] = f32_to_bf16_bits(x)
-        del x
-    out["A_log"] = rng.standard_normal(size=(w.Nv,), dtype=np.float32)
-    out["dt_bias"] = rng.standard_normal(size=(w.Nv, w.D), dtype=np.float32)
+    for stream, (name, key) in enumerate((("q", "q"), ("k", "q"), ("v", "v"), ("g", "v"),
+                                          ("beta", "beta"))):
+        out[name] = f32_to_bf16_bits(normal_f32(w.seed, stream, sh[key]))
+    out["A_log"] = normal_f32(w.seed, 5, (w.Nv,))
+    out["dt_bias"] = normal_f32(w.seed, 6, (w.Nv, w.D))
     if w.init_state == "zeros":
         out["initial_state"] = np.zeros((w.B, w.Nv, w.D, w.D), dtype=np.float32)
     else:
-        out["initial_state"] = (rng.standard_normal(size=(w.B, w.Nv, w.D, w.D), dtype=np.float32)
-                                * np.float32(w.init_std))
+        out["initial_state"] = normal_f32(w.seed, 7, (w.B, w.Nv, w.D, w.D)) * np.float32(w.init_std)
     out["cu_seqlens"] = w.cu_seqlens
     if pad_value is not None and w.layout != "TND":
         pv = f32_to_bf16_bits(np.array([pad_value], dtype=np.float32))[0]
