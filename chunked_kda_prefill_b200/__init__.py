@@ -6,6 +6,6 @@ the thin Python binding over it.  Build the library with
 """
 from ._lib import EXPORTS, LIB_PATH, KdaError, KdaShape, load  # noqa: F401
 from .api import (KdaPlan, LAYOUTS, decode, device_status, flash_kda, flash_kda_noalloc,  # noqa: F401
-                  forward_kernel_names, forward_summary, kernels_per_forward, make_plan, plan,
-                  state_chain)
+                  forward_kernel_names, forward_summary, kernels_per_forward, make_plan,
+                  noalloc_status, plan, state_chain)
 from .context_parallel import flash_kda_context_parallel  # noqa: F401

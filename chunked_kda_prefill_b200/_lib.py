@@ -12,7 +12,7 @@ LIB_PATH = os.environ.get("KDA_LIB") or os.path.join(PKG, "libkda.so")
 # Every symbol include/kda.h declares.
 EXPORTS = ("kda_status_string", "kda_plan_size", "kda_plan", "kda_workspace_size",
            "kda_forward", "kda_device_status", "kda_forward_noalloc", "kda_decode",
-           "kda_plan_segmented", "kda_forward_summary", "kda_state_chain")
+           "kda_plan_segmented", "kda_forward_summary", "kda_state_chain", "kda_noalloc_status")
 
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_NULL", 2: "KDA_ERR_LAYOUT", 3: "KDA_ERR_SHAPE",
           4: "KDA_ERR_HEADS", 5: "KDA_ERR_DIM", 6: "KDA_ERR_LOWER_BOUND", 7: "KDA_ERR_SEQLENS",
@@ -60,6 +60,7 @@ def load():
     L.kda_device_status.argtypes = [vp, vp]
     L.kda_forward_noalloc.argtypes = [p_shape, p_i32, vp, sz, vp, vp, vp, vp, vp, ctypes.c_float,
                                       vp, vp, vp, ctypes.c_float, vp, vp, vp]
+    L.kda_noalloc_status.argtypes = [vp]
     L.kda_plan_segmented.argtypes = [p_shape, p_i32, i32, i32, p_i32, sz]
     L.kda_decode.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
                              ctypes.c_float, vp, vp, vp]
@@ -68,7 +69,7 @@ def load():
     L.kda_state_chain.argtypes = [i32, i32, i32, vp, vp, vp, ctypes.c_int64, vp, vp]
     for f in ("kda_plan_size", "kda_plan", "kda_workspace_size", "kda_forward",
               "kda_device_status", "kda_forward_noalloc", "kda_decode", "kda_plan_segmented",
-              "kda_forward_summary", "kda_state_chain"):
+              "kda_forward_summary", "kda_state_chain", "kda_noalloc_status"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L

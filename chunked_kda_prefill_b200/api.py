@@ -217,7 +217,8 @@ def flash_kda_noalloc(q, k, v, g, beta, scale: float, initial_state, A_log, dt_b
     """flash_kda through kda_forward_noalloc: no workspace, the library's fixed scratch instead.
 
     For callers that cannot allocate device memory; the caller still provides out and
-    final_state.  Raises KdaError(KDA_ERR_CAPACITY) for problems larger than the scratch.
+    final_state.  It runs the same kernels as flash_kda.  Raises KdaError(KDA_ERR_CAPACITY) for
+    a plan whose workspace would exceed the scratch.  noalloc_status() reads the device status.
     """
     dev = q.device
     if out is None or final_state is None:
@@ -350,6 +351,15 @@ def device_status(workspace: torch.Tensor, stream: torch.cuda.Stream | None = No
     """Synchronise and raise if the last forward on this workspace recorded a device error."""
     s = stream if stream is not None else torch.cuda.current_stream(workspace.device)
     check(_lib.load().kda_device_status(workspace.data_ptr(), s.cuda_stream), "kda_device_status")
+
+
+def noalloc_status(device=None, stream: torch.cuda.Stream | None = None) -> None:
+    """Synchronise and raise if the last flash_kda_noalloc on this device recorded a device
+    error (its status word lives in the library's fixed scratch)."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        check(_lib.load().kda_noalloc_status(s.cuda_stream), "kda_noalloc_status")
 
 
 def kernels_per_forward(plan: KdaPlan | None = None) -> int:

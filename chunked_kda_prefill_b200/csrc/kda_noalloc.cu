@@ -58,16 +58,25 @@ extern "C" kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int3
   if (!plan_host) return KDA_ERR_NULL;
   st = validate_plan(plan_host, n_int32, shape);
   if (st != KDA_OK) return st;
-  const size_t need = simt_workspace_bytes(plan_host);
+  const size_t need = fused_workspace_bytes(plan_host);
   if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_CAPACITY;
   void* scratch = nullptr;
   st = scratch_on_current_device(&scratch);
   if (st != KDA_OK) return st;
-  // The two-kernel path: the per-chunk intermediates live in the scratch.  The status word at
-  // its start is cleared on every call; every other byte the kernels read is written earlier in
-  // the same call.
-  return forward_impl(PATH_SIMT, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
+  // Exactly kda_forward, with the scratch as its workspace: the device status word at its start
+  // is cleared on every call, and under a segmented plan the segment state slots that follow it
+  // are written before they are read within the same call.
+  return forward_impl(PATH_FUSED, shape, plan_host, plan_dev, n_int32, q, k, v, g, beta, scale,
                       initial_state, A_log, dt_bias, lower_bound, scratch,
                       (size_t)KDA_NOALLOC_SCRATCH_BYTES, out, final_state,
                       reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+// The device status word of the last kda_forward_noalloc on the current device: it lives at the
+// start of that device's scratch, so this is kda_device_status on the scratch.
+extern "C" kda_status_t kda_noalloc_status(kda_stream_t stream) {
+  void* scratch = nullptr;
+  const kda_status_t st = scratch_on_current_device(&scratch);
+  if (st != KDA_OK) return st;
+  return kda_device_status(scratch, stream);
 }

@@ -94,10 +94,13 @@ KDA_API kda_status_t kda_plan_size(const kda_shape_t* shape, size_t* n_int32);
 
 /* Build the schedule (the flash_kda_metadata equivalent, FlashKDA README 功能说明: built from
  * shapes, layout, valid lengths and the device's core count; reads no tensor values).
- *   cu_seqlens_host: host int32 [B+1] prefix sums of the valid lengths.
- *     TND : required; cu[0] == 0, cu[B] == T, strictly increasing.
- *     BNSD/BSND: optional (NULL = every length is S); each length cu[b+1]-cu[b] in [1, S];
+ *   cu_seqlens_host: host int32 [B+1], in every layout the prefix sums of the valid lengths:
+ *     cu[0] == 0 and len_b = cu[b+1] - cu[b] >= 1, so the array is strictly increasing and
+ *     cu[B] is the sum of the lengths.
+ *     TND : required, and cu[B] == T (the packed row count).
+ *     BNSD/BSND: optional (NULL = every length is S); each len_b is also <= S, so cu[B] <= B*S;
  *     sequence b then occupies storage rows [0, len_b) of slot b (FlashKDA README 约束说明).
+ *     Anything else is KDA_ERR_SEQLENS.
  *   num_sms: multiprocessor count of the target device (>= 1); recorded in the plan.
  *   plan, n_int32: host output buffer and its capacity in int32 words.
  * Units are ordered longest first.  Pure host code; never touches the GPU.
@@ -215,20 +218,21 @@ KDA_API kda_status_t kda_device_status(const void* workspace, kda_stream_t strea
  * interface that hands over only the tensors, or a host runtime whose memory pool forbids
  * extra cudaMalloc calls (cudaMalloc can also synchronise the device).
  *
- * Arguments, layouts and results are those of kda_forward, without workspace and
- * workspace_bytes.  Instead the library uses one fixed scratch array of
- * KDA_NOALLOC_SCRATCH_BYTES per GPU: a static __device__ array that every GPU loading libkda.so
- * holds until the process exits.  The call allocates nothing (no cudaMalloc, cudaFree or
- * allocating library routine).
- *   - Problems whose kda_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES are rejected with
- *     KDA_ERR_CAPACITY before anything is enqueued (the current kernels need 148,480 bytes per
- *     64-token chunk of every (sequence, value head), plus 256, so at most 451 such chunks).
+ * It runs exactly what kda_forward runs (the same kernels, schedule and results, D = 128 or
+ * 64), with the same arguments minus workspace and workspace_bytes.  In place of the caller's
+ * workspace the library uses one fixed scratch array of KDA_NOALLOC_SCRATCH_BYTES per GPU: a
+ * static __device__ array that every GPU loading libkda.so holds until the process exits.  The
+ * call allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - A plan whose kda_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES is rejected with
+ *     KDA_ERR_CAPACITY before anything is enqueued.  A whole-unit plan needs 256 bytes; a
+ *     segmented plan adds 196,608 bytes per segment after each unit's first, so up to 341 such
+ *     segments fit.
  *   - The first call on each device looks up the scratch's device address with that device
  *     current and caches it; make that first call before any stream capture.
  *   - Every call on a device shares the one scratch array, which keeps the last call's contents
  *     (the call clears what must start at zero).  Calls whose kernels overlap on the GPU (two
  *     streams, or two host threads) race on it: serialise them.
- *   - The device status word lives in that scratch; there is no kda_device_status for it. */
+ *   - The device status word lives at the start of the scratch: kda_noalloc_status reads it. */
 KDA_API kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int32_t* plan_host,
                                          const int32_t* plan_dev, size_t n_int32, const void* q,
                                          const void* k, const void* v, const void* g,
@@ -236,6 +240,11 @@ KDA_API kda_status_t kda_forward_noalloc(const kda_shape_t* shape, const int32_t
                                          const float* initial_state, const float* A_log,
                                          const float* dt_bias, float lower_bound, void* out,
                                          float* final_state, kda_stream_t stream);
+
+/* kda_device_status for kda_forward_noalloc: synchronise `stream` and return the device-side
+ * status recorded in the current device's fixed scratch by the last kda_forward_noalloc there
+ * (KDA_OK, KDA_ERR_PLAN or KDA_ERR_TIMEOUT), or KDA_ERR_CUDA.  Allocates nothing. */
+KDA_API kda_status_t kda_noalloc_status(kda_stream_t stream);
 
 /* The single-token decode step that follows a prefill: one step of the recurrence the chunked
  * forward computes in 64-token blocks (FlashKDA README, 功能说明; FLA PR 656, "[kda] add
