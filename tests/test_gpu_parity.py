@@ -1,5 +1,7 @@
 """CUDA path vs the fp64 oracle, element by element (atol = rtol = 5e-3), plus bookkeeping that
 must be bit-exact (layouts, varlen packing, GQA, padding, chaining, determinism)."""
+import os
+
 import numpy as np
 import pytest
 
@@ -33,9 +35,29 @@ def test_workload_full_parity(idx, cuda_ok):
 
 
 @pytest.mark.parametrize("idx", [4, 5, 7])
+def test_workload_every_unit_parity(idx, cuda_ok):
+    """Full-size run (the benchmarked launch) against the oracle on every (sequence, head) unit,
+    element by element: out on every valid row and every final state.  The oracle runs its
+    token-by-token form (pinned equal to the chunked form) on all host threads.  Workload 7 takes
+    the segmented schedule by default, so this covers that schedule at full size."""
+    w = W.workload(idx)
+    inp = W.generate(w)
+    o_g, fs_g = run_gpu(w, inp)
+    res = oracle.run_units(inp, w.layout, w.B, w.Nqk, w.Nv, w.S, w.D, w.scale, w.lower_bound,
+                           w.cu_seqlens, form="recurrent", threads=os.cpu_count())
+    assert len(res) == w.B * w.Nv
+    for (b, h), (o_r, fs_r) in res.items():
+        compare(unit_rows(w, o_g, b, h), o_r, f"{w.name} out ({b},{h})")
+        compare(fs_g[b, h], fs_r, f"{w.name} final_state ({b},{h})")
+    m = valid_mask(w, o_g.shape)
+    assert np.all(o_g[~m] == 0.0)
+    assert np.all(np.isfinite(o_g)) and np.all(np.isfinite(fs_g))
+
+
+@pytest.mark.parametrize("idx", [4, 5, 7])
 def test_workload_sampled_parity(idx, cuda_ok):
-    """Full-size run (the benchmarked launch), oracle on a sample of whole units.  Workload 7
-    takes the segmented schedule by default, so this is that schedule at full size."""
+    """Quick variant of the above: the chunked oracle on a sample of whole units (first, last,
+    longest and shortest sequence; first and last head)."""
     w = W.workload(idx)
     inp = W.generate(w)
     o_g, fs_g = run_gpu(w, inp)
@@ -47,9 +69,6 @@ def test_workload_sampled_parity(idx, cuda_ok):
     for (b, h), (o_r, fs_r) in res.items():
         compare(unit_rows(w, o_g, b, h), o_r, f"{w.name} out ({b},{h})")
         compare(fs_g[b, h], fs_r, f"{w.name} final_state ({b},{h})")
-    m = valid_mask(w, o_g.shape)
-    assert np.all(o_g[~m] == 0.0)
-    assert np.all(np.isfinite(o_g)) and np.all(np.isfinite(fs_g))
 
 
 SMALL = [
