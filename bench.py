@@ -160,8 +160,10 @@ def ncu_traffic(workload_name: str):
 # CPU oracle baseline (bounded sample)
 # ----------------------------------------------------------------------------
 
-def cpu_oracle_sample(w: W.Workload, inp: dict, budget_s: float = 10.0, tokens: int | None = None):
-    """Time the fp64 oracle (recurrence) on batches of whole units until ``budget_s`` elapses.
+def cpu_oracle_sample(w: W.Workload, inp: dict, budget_s: float = 10.0, tokens: int | None = None,
+                      form: str = "recurrent"):
+    """Time the fp64 oracle (``form``: the recurrence, or the chunked form) on batches of whole
+    units until ``budget_s`` elapses.
 
     One batch is one unit per host thread.  ``tokens`` keeps only the first ``tokens`` rows of
     every sequence (BNSD/BSND), a bounded sample with the same per-token work.
@@ -183,7 +185,7 @@ def cpu_oracle_sample(w: W.Workload, inp: dict, budget_s: float = 10.0, tokens: 
         batch = units[i:i + cores]
         i += cores
         oracle.run_units(it, w.layout, w.B, w.Nqk, w.Nv, S, w.D, w.scale, w.lower_bound, cu,
-                         units=batch, form="recurrent", threads=cores)
+                         units=batch, form=form, threads=cores)
         done_tokens += sum(lengths[b] for b, _ in batch)
         n_units += len(batch)
         if time.perf_counter() - t0 >= budget_s:
@@ -192,7 +194,8 @@ def cpu_oracle_sample(w: W.Workload, inp: dict, budget_s: float = 10.0, tokens: 
     return {"value": done_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n_units} whole (sequence, value head) units of {w.name}"
                       + ("" if tokens is None else f", first {tokens} tokens each")
-                      + f", fp64 recurrence, {dt:.1f} s wall on {cores} threads"}, dt
+                      + (", fp64 recurrence" if form == "recurrent" else ", fp64 chunked form")
+                      + f", {dt:.1f} s wall on {cores} threads"}, dt
 
 
 # ----------------------------------------------------------------------------
@@ -404,11 +407,97 @@ def run_ours(args, rank, world):
                          "tensor_tflops": algorithmic_flops(w) / (kernel_ms / 1e3) / 1e12}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"], _ = cpu_oracle_sample(w, inp, budget_s=args.cpu_budget)
+    if rank == 0 and world == 1 and not args.no_per_config:
+        del d, out, fs, ws
+        if not args.no_e2e:
+            del bufs
+        torch.cuda.empty_cache()
+        line["per_config"] = per_config(args, dev, kda, cached=(args.workload, inp))
     if dist is not None:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+PER_CONFIG = (1, 2, 3, 4, 5, 6, 7)
+
+
+def time_calls(fn, n: int, stream, flush=None) -> list:
+    """Device time of each of n calls of fn, each bracketed by its own CUDA events on `stream`;
+    `flush` (a buffer larger than L2) is zeroed before every call, outside the brackets."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            if flush is not None:
+                flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def per_config(args, dev, kda, cached=None):
+    """Every synthetic workload on this GPU: the median and p10/p90 of --per-config-calls calls
+    (each timed alone, after 10 warm-up calls; L2 flushed before each call when the inputs fit
+    in it), token-heads/s and the HBM roofline fraction at the median, the schedule, and the
+    fp64 oracle's token-heads/s in both forms on a bounded sample, with its thread count."""
+    import torch
+    peak, peak_kind = measured_peaks()
+    rows = []
+    for idx in PER_CONFIG:
+        w = W.workload(idx)
+        inp = cached[1] if cached is not None and cached[0] == idx else W.generate(w)
+        d = {n: torch.from_numpy(np.ascontiguousarray(inp[n]).view(np.int16)).view(
+            torch.bfloat16).to(dev) for n in ("q", "k", "v", "g", "beta")}
+        for n in ("A_log", "dt_bias", "initial_state"):
+            d[n] = torch.from_numpy(np.ascontiguousarray(inp[n], dtype=np.float32)).to(dev)
+        cu = w.cu_seqlens if (w.layout == "TND" or any(L != w.S for L in w.lengths)) else None
+        plan = kda.plan(d["q"], d["v"], d["initial_state"], w.layout, cu_seqlens=cu)
+        ws = plan.workspace()
+        out = torch.empty_like(d["v"])
+        fs = torch.empty((w.B, w.Nv, w.D, w.D), dtype=torch.float32, device=dev)
+        stream = torch.cuda.Stream(dev)
+        in_bytes = 5 * (w.S if w.layout == "TND" else w.B * w.S) * w.Nv * w.D * 2
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes <= 126e6 else None
+
+        def fwd():
+            kda.flash_kda(d["q"], d["k"], d["v"], d["g"], d["beta"], w.scale, d["initial_state"],
+                          d["A_log"], d["dt_bias"], w.lower_bound, w.layout, plan, out=out,
+                          final_state=fs, workspace=ws, stream=stream)
+
+        time_calls(fwd, 10, stream, flush)
+        ms = np.array(time_calls(fwd, args.per_config_calls, stream, flush))
+        kda.device_status(ws, stream)
+        med = float(np.median(ms))
+        abytes = algorithmic_bytes(w, True)
+        row = {"workload": w.name, "calls": int(ms.size), "ms_median": med,
+               "ms_p10": float(np.percentile(ms, 10)), "ms_p90": float(np.percentile(ms, 90)),
+               "token_heads": w.token_heads, "value": w.token_heads / (med / 1e3), "unit": UNIT,
+               "roofline": {"bound": "hbm", "achieved": abytes / (med / 1e3) / 1e9,
+                            "peak": peak, "unit": "GB/s",
+                            "frac": abytes / (med / 1e3) / 1e9 / peak,
+                            "peak_source": f"{peak_kind} hbm_gbs",
+                            "algorithmic_bytes": abytes},
+               "schedule": (f"segments of {plan.segment_chunks} chunks"
+                            if plan.segment_chunks > 0 else "whole units"),
+               "l2": "flushed before each call" if flush is not None else "inputs larger than L2"}
+        del d, out, fs, ws, plan, flush
+        torch.cuda.empty_cache()
+        if not args.no_cpu_baseline:
+            row["oracle"] = {}
+            for form in ("recurrent", "chunked"):
+                r, _ = cpu_oracle_sample(w, inp, budget_s=args.per_config_cpu_budget,
+                                         tokens=min(w.S, 2048) if w.layout != "TND" else None,
+                                         form=form)
+                row["oracle"][form] = {"value": r["value"], "unit": UNIT, "cores": r["cores"],
+                                       "sample": r["sample"]}
+        rows.append(row)
+        del inp
+    return rows
 
 
 def rank_workload(idx: int, rank: int, world: int) -> W.Workload:
@@ -623,6 +712,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload table (workloads 1-7, rank 0 at N = 1 only)")
+    ap.add_argument("--per-config-calls", type=int, default=50)
+    ap.add_argument("--per-config-cpu-budget", type=float, default=1.5,
+                    help="seconds of oracle time per workload and form")
     ap.add_argument("--mode", default="prefill", choices=["prefill", "decode", "cp"],
                     help="prefill (the default, the headline), the single-token decode step, "
                          "or context parallelism (one sequence split over the ranks)")
@@ -636,6 +730,7 @@ def main():
                          "chunks (chunk-parallel scan)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.per_config_calls = max(args.per_config_calls, 50)
     rank = _env_int("RANK", 0)
     world = _env_int("WORLD_SIZE", 1)
     if args.impl == "reference":
