@@ -12,8 +12,9 @@
 //   2 MMA  D_I = Aop B^(I)^T, I = 0..3 (M=128, N=160 for all four blocks, K=128): rows 0-63 give
 //     T = stril(diag(beta) K~ K-^T), rows 64-127 give Aqk = tril(Q~ K-^T); meanwhile K^ lo is
 //     stored and the state left by the previous chunk becomes the bf16 hi/lo state operand
-//   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 16x16 diagonal blocks and two merge levels;
-//     Xsol = X diag(beta) -> bf16 hi and lo parts stacked as one 128-row operand
+//   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 16x16 blocks (diagonal inverses in registers,
+//     then rounds of independent block products); Xsol = X diag(beta) -> bf16 hi and lo parts
+//     stacked as one 128-row operand
 //   4 MMA  W^T = K~^T [Xsol_hi; Xsol_lo]^T and U^T = V^T [Xsol_hi; Xsol_lo]^T (one N=128 chain
 //          each, hi and lo parts side by side); S <- S Diag(2^G_last)
 //     meanwhile.  Then -W -> bf16 hi and lo, stored token-major over the K~ and V tiles
@@ -50,12 +51,6 @@ using namespace sm100;
 
 constexpr int kThreads = 512;
 
-// Variants of the first level of the triangular solve, for the solve ablation (build with
-// -DKDA_SOLVE_L1=n): 0 = 8x8 diagonal inverses + 8->16 merges, CTA-wide (default, fastest);
-// 1 = 16x16 column substitution; 2 = 8x8 + merge warp-local.
-#ifndef KDA_SOLVE_L1
-#define KDA_SOLVE_L1 0
-#endif
 // The state operand of phase 5: a bf16 hi/lo pair (1, default) or the bf16 hi part alone (0: no
 // lo conversion and 8 fewer MMAs per chunk, at a lower precision of W S^T and Q~ S^T; a variant
 // for precision/speed experiments, built with -DKDA_STATE_LO=0).
@@ -108,7 +103,8 @@ constexpr uint32_t SM_END = 230304;
 constexpr size_t kFusedSmemBytes = SM_END + 1024;
 
 // per-(block, column) constants of the operand factorisation, indices into SM_CST
-enum : int { CST_REF = 0, CST_GE, CST_P2REF, CST_KFAC, CST_CDIAG, CST_C2, CST_C3, CST_N };
+// (CST_NREF holds the reference row's cumulative gate negated, so that phase 1 adds it)
+enum : int { CST_NREF = 0, CST_GE, CST_P2REF, CST_KFAC, CST_CDIAG, CST_C2, CST_C3, CST_N };
 
 // Phase timestamps for performance analysis (CTA 0, thread 0, first 64 chunks), compiled in
 // only for a profiling build (-DKDA_PHASE_TIMING=1): every thread would otherwise evaluate the
@@ -126,6 +122,53 @@ enum : int { CST_REF = 0, CST_GE, CST_P2REF, CST_KFAC, CST_CDIAG, CST_C2, CST_C3
   do {                \
   } while (0)
 #endif
+
+// The triangular solve's rounds of 16x16 block products (phase 3): O = C + sg (L R), operands
+// as float offsets from the shared-memory base.  T and X are [64][kSolveTP] fp32 in the B-tile
+// region (free after the intra MMA), twelve scratch blocks Z0..Z11 [16][kSolveBP] in the upper
+// half of the Aop region; xi >= 0 marks a final block X_(xi,xj), also written out as Xsol.
+constexpr int kSolveTP = 68, kSolveBP = 20;
+struct SolveOp {
+  uint16_t l, ldl, r, ldr, c, ldc, o, ldo;  // offsets (floats) and row pitches
+  int8_t sg;                                 // sg == 0: no product;  c == 0: no C term
+  int8_t xi, xj, pad;
+};
+constexpr int kTs = (int)(SM_BT / 4), kXs = kTs + 64 * kSolveTP, kZs = (int)((SM_AOP + 16384) / 4);
+static_assert(kXs + 64 * kSolveTP <= (int)(SM_KLO / 4), "T and X overflow the B-tile region");
+static_assert(12 * 16 * kSolveBP <= 16384 / 4, "scratch blocks overflow the Aop upper half");
+static_assert(kZs + 12 * 16 * kSolveBP < 65536, "offsets must fit 16 bits");
+constexpr uint16_t TBo(int I, int J) { return (uint16_t)(kTs + 16 * I * kSolveTP + 16 * J); }
+constexpr uint16_t XBo(int I, int J) { return (uint16_t)(kXs + 16 * I * kSolveTP + 16 * J); }
+constexpr uint16_t ZBo(int z) { return (uint16_t)(kZs + z * 16 * kSolveBP); }
+constexpr uint16_t TPs = kSolveTP, BPs = kSolveBP;
+constexpr SolveOp kNoOp = {0, 0, 0, 0, 0, 0, 0, 0, 0, -1, 0, 0};
+__constant__ SolveOp kSolveOps[4][8] = {
+    {// R2: A_IJ = T_IJ P_J -> Z0..Z5;  G21 = -P2 T21 -> Z6;  G31 = -P3 T31 -> Z7
+     {TBo(1, 0), TPs, XBo(0, 0), TPs, 0, 0, ZBo(0), BPs, 1, -1, 0, 0},
+     {TBo(2, 1), TPs, XBo(1, 1), TPs, 0, 0, ZBo(1), BPs, 1, -1, 0, 0},
+     {TBo(3, 2), TPs, XBo(2, 2), TPs, 0, 0, ZBo(2), BPs, 1, -1, 0, 0},
+     {TBo(2, 0), TPs, XBo(0, 0), TPs, 0, 0, ZBo(3), BPs, 1, -1, 0, 0},
+     {TBo(3, 1), TPs, XBo(1, 1), TPs, 0, 0, ZBo(4), BPs, 1, -1, 0, 0},
+     {TBo(3, 0), TPs, XBo(0, 0), TPs, 0, 0, ZBo(5), BPs, 1, -1, 0, 0},
+     {XBo(2, 2), TPs, TBo(2, 1), TPs, 0, 0, ZBo(6), BPs, -1, -1, 0, 0},
+     {XBo(3, 3), TPs, TBo(3, 1), TPs, 0, 0, ZBo(7), BPs, -1, -1, 0, 0}},
+    {// R3: X10, X21, X32 = -P_I A_IJ;  D20, D31, D30 = -P_I A_IJ -> Z8..Z10;  G32 -> Z11
+     {XBo(1, 1), TPs, ZBo(0), BPs, 0, 0, XBo(1, 0), TPs, -1, 1, 0, 0},
+     {XBo(2, 2), TPs, ZBo(1), BPs, 0, 0, XBo(2, 1), TPs, -1, 2, 1, 0},
+     {XBo(3, 3), TPs, ZBo(2), BPs, 0, 0, XBo(3, 2), TPs, -1, 3, 2, 0},
+     {XBo(2, 2), TPs, ZBo(3), BPs, 0, 0, ZBo(8), BPs, -1, -1, 0, 0},
+     {XBo(3, 3), TPs, ZBo(4), BPs, 0, 0, ZBo(9), BPs, -1, -1, 0, 0},
+     {XBo(3, 3), TPs, ZBo(5), BPs, 0, 0, ZBo(10), BPs, -1, -1, 0, 0},
+     {XBo(3, 3), TPs, TBo(3, 2), TPs, 0, 0, ZBo(11), BPs, -1, -1, 0, 0},
+     kNoOp},
+    {// R4: X20 = D20 + G21 X10;  X31 = D31 + G32 X21;  E30 = D30 + G31 X10 -> Z0
+     {ZBo(6), BPs, XBo(1, 0), TPs, ZBo(8), BPs, XBo(2, 0), TPs, 1, 2, 0, 0},
+     {ZBo(11), BPs, XBo(2, 1), TPs, ZBo(9), BPs, XBo(3, 1), TPs, 1, 3, 1, 0},
+     {ZBo(7), BPs, XBo(1, 0), TPs, ZBo(10), BPs, ZBo(0), BPs, 1, -1, 0, 0},
+     kNoOp, kNoOp, kNoOp, kNoOp, kNoOp},
+    {// R5: X30 = E30 + G32 X20
+     {ZBo(11), BPs, XBo(2, 0), TPs, ZBo(0), BPs, XBo(3, 0), TPs, 1, 3, 0, 0},
+     kNoOp, kNoOp, kNoOp, kNoOp, kNoOp, kNoOp, kNoOp}};
 
 __device__ __forceinline__ uint32_t dcol(int I) { return 8u * I * (I + 1); }
 
@@ -159,6 +202,24 @@ __device__ __forceinline__ uint32_t split_lo(float a, float b, uint32_t hi) {
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
+}
+
+// fp32 -> tf32 (round to nearest, ties away; the low 13 mantissa bits cleared)
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+// d += a b for one 16x8x8 tile on the warp-level tensor-core path (tf32 inputs, fp32 d), with
+// the PTX fragment layouts: a = A(g, t), A(g+8, t), A(g, t+4), A(g+8, t+4); b = B(t, g), B(t+4, g);
+// d = D(g, 2t), D(g, 2t+1), D(g+8, 2t), D(g+8, 2t+1), where g = lane / 4 and t = lane % 4.
+__device__ __forceinline__ void mma_tf32_m16n8k8(float (&d)[4], const uint32_t (&a)[4],
+                                                 const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 struct Maps {
@@ -361,8 +422,9 @@ template <int DIM, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_kernel(const Params p, const __grid_constant__ Maps maps, float* dbg) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
+  // 1024-byte aligned base, by an offset into the shared array itself (not through an integer
+  // round trip) so that the compiler keeps every access below in the shared state space
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // K steps of 16 over the head dim in the MMAs that contract it (phases 2 and 5): at D = 64 the
@@ -547,33 +609,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       // rows 4 grp .. 4 grp + 3; warp 0 issues the MMAs this overlaps, so warp 4 (the same SM
       // sub-partition) takes its rows as well
       auto group = [&](int grp) {
-        float G[4][4];
+        float2 G[4][2];  // rows x column pairs (packed fp32x2 arithmetic)
+        const float2 ca2 = make_float2(ca, ca), one2 = make_float2(1.f, 1.f);
+        const float2 lb2 = make_float2(lbl2, lbl2);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = 4 * grp + i;
-          float gv[4];
           // (row 4 grp + i has the swizzle of row r0 + i: grp and warp have the same parity)
           const int off = (int)(colhalf * QGV_ATOM + io[i]) + (grp - warp) * 512;
-          unpack4(*reinterpret_cast<const uint2*>(sg_tile + off), gv);
+          const uint2 w = *reinterpret_cast<const uint2*>(sg_tile + off);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float sgm = __fdividef(lbl2, 1.0f + ex2(ca * (gv[e] + dtb[e])));
-            G[i][e] = (r < nn) ? sgm : 0.0f;
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t wh = h ? w.y : w.x;
+            const float2 x = __fmul2_rn(
+                __fadd2_rn(make_float2(bf16_lo_of(wh), bf16_hi_of(wh)),
+                           make_float2(dtb[2 * h], dtb[2 * h + 1])), ca2);
+            const float2 den = __fadd2_rn(make_float2(ex2(x.x), ex2(x.y)), one2);
+            const float2 sgm = __fmul2_rn(make_float2(__fdividef(1.0f, den.x),
+                                                      __fdividef(1.0f, den.y)), lb2);
+            G[i][h] = (r < nn) ? sgm : make_float2(0.f, 0.f);
           }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          if (i > 0)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) G[i][e] += G[i - 1][e];
+          if (i > 0) {
+            G[i][0] = __fadd2_rn(G[i][0], G[i - 1][0]);
+            G[i][1] = __fadd2_rn(G[i][1], G[i - 1][1]);
+          }
           *reinterpret_cast<float4*>(gtile + (4 * grp + i) * kD + j0) =
-              make_float4(G[i][0], G[i][1], G[i][2], G[i][3]);
+              make_float4(G[i][0].x, G[i][0].y, G[i][1].x, G[i][1].y);
         }
         *reinterpret_cast<float4*>(wtot + grp * kD + j0) =
-            make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+            make_float4(G[3][0].x, G[3][0].y, G[3][1].x, G[3][1].y);
       };
-      if (warp != 0) group(warp);
-      if (warp == 4) group(0);
+      // (one call site: warp 4 runs it twice)
+#pragma unroll 1
+      for (int rep = (warp == 4) ? 0 : 1; rep < 2; ++rep)
+        if (warp != 0) group(rep == 0 ? 0 : warp);
       if (tid >= kChunk && tid < 2 * kChunk)  // (beta: threads 64-127, not warp 0)
         beta_s[tid - kChunk] =
             (tid - kChunk < nn) ? __fdividef(1.0f, 1.0f + __expf(-__bfloat162float(blog))) : 0.0f;
@@ -597,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int I = 0; I < 4; ++I) {
         const float refI = (I == 0) ? 0.f : ref[I - 1];
         const float ge = ref[I];
-        cst[(CST_REF * 4 + I) * kD + j] = refI;
+        cst[(CST_NREF * 4 + I) * kD + j] = -refI;
         cst[(CST_GE * 4 + I) * kD + j] = ge;
         cst[(CST_P2REF * 4 + I) * kD + j] = ex2(refI);
         cst[(CST_KFAC * 4 + I) * kD + j] = ex2(ref[3] - ge);
@@ -711,66 +783,65 @@ __global__ void __launch_bounds__(kThreads, 1)
             rkv[m] = __shfl_sync(0xffffffffu, y, 16 + 4 * (m & 1) + 8 * (m >> 1));
           }
         }
-        // the rows of this warp's 16-row block JB (warp-uniform) as a compile-time constant, so
-        // the staircase copies B^(JB..3) need no runtime block arithmetic or branches
-        auto rows = [&](auto jb_const) {
-          constexpr int JB = decltype(jb_const)::value;
+        // this thread's 4 rows x 4 columns as two fp32 pairs per row (packed fp32x2 arithmetic);
+        // the staircase copies B^(Jb..3) of the warp's 16-row block Jb (warp-uniform)
+        auto f2 = [](float a, float b) { return make_float2(a, b); };
+        const float2 m1 = f2(-1.f, -1.f);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = r0 + i;
-            const bool valid = r < n;
-            float qv[4], kv[4];
-            unpack4(qwv[i], qv);
-            unpack4(kwv[i], kv);
-            const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
-            const float rk = rsqrtf(rkv[i] + 1e-6f);
-            float ka[4], qa[4], kt[4], qt[4], kh[4], b0[4], b1[4], b2[4], b3[4];
+        for (int i = 0; i < 4; ++i) {
+          const int r = r0 + i;
+          const bool valid = r < n;
+          const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
+          const float rk = rsqrtf(rkv[i] + 1e-6f);
+          const float2 rq2 = f2(rq, rq), rk2 = f2(rk, rk);
+          uint32_t pa[2], pq[2], pqt[2], pkh[2], pkt[2], pb0[2], pb1[2], pb2[2], pb3[2], pkl[2];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float Gv = G[i][e];
-              const float kn = kv[e] * rk;
-              const float qn = qv[e] * rq;
-              const float fA = ex2(Gv - k4[CST_REF][e]);
-              const float kbe = kn * ex2(k4[CST_GE][e] - Gv);
-              ka[e] = kn * fA;
-              qa[e] = qn * fA;
-              kt[e] = ka[e] * k4[CST_P2REF][e];
-              qt[e] = qa[e] * k4[CST_P2REF][e];
-              kh[e] = kbe * k4[CST_KFAC][e];
-              b0[e] = kbe * k4[CST_CDIAG][e];  // B^(Jb): diagonal block
-              b1[e] = kbe;                     // B^(Jb+1): reference row is this block's last row
-              if (JB + 2 <= 3) b2[e] = kbe * k4[CST_C2][e];  // B^(Jb+2)
-              if (JB + 3 <= 3) b3[e] = kbe * k4[CST_C3][e];  // B^(Jb+3)
-            }
-            const uint2 khp = pack4(kh[0], kh[1], kh[2], kh[3]);
-            khlo[i] = make_uint2(split_lo(kh[0], kh[1], khp.x), split_lo(kh[2], kh[3], khp.y));
-            uint8_t* aop = sm + SM_AOP + colhalf * 16384u + io[i];
-            uint8_t* bst = sm + SM_BT + colhalf * (BT_ROWS * 128u) + io[i];
-            *reinterpret_cast<uint2*>(aop) = pack4(ka[0], ka[1], ka[2], ka[3]);
-            *reinterpret_cast<uint2*>(aop + 8192) = pack4(qa[0], qa[1], qa[2], qa[3]);
-            *reinterpret_cast<uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]) = pack4(qt[0], qt[1], qt[2], qt[3]);
-            *reinterpret_cast<uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]) = khp;
-            *reinterpret_cast<uint2*>(sq + OFF_G + colhalf * QGV_ATOM + io[i]) = pack4(kt[0], kt[1], kt[2], kt[3]);
-            *reinterpret_cast<uint2*>(bst + dcol(JB) * 128u) =
-                pack4(b0[0], b0[1], b0[2], b0[3]);
-            if (JB + 1 <= 3)
-              *reinterpret_cast<uint2*>(bst + dcol(JB + 1) * 128u) =
-                  pack4(b1[0], b1[1], b1[2], b1[3]);
-            if (JB + 2 <= 3)
-              *reinterpret_cast<uint2*>(bst + dcol(JB + 2) * 128u) =
-                  pack4(b2[0], b2[1], b2[2], b2[3]);
-            if (JB + 3 <= 3)
-              *reinterpret_cast<uint2*>(bst + dcol(JB + 3) * 128u) =
-                  pack4(b3[0], b3[1], b3[2], b3[3]);
-            if (!valid || it.zero_v)  // an M run treats v as zero
-              *reinterpret_cast<uint2*>(sq + OFF_V + colhalf * QGV_ATOM + io[i]) = make_uint2(0, 0);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t kw = h ? kwv[i].y : kwv[i].x, qw = h ? qwv[i].y : qwv[i].x;
+            const float2 kv2 = f2(bf16_lo_of(kw), bf16_hi_of(kw));
+            const float2 qv2 = f2(bf16_lo_of(qw), bf16_hi_of(qw));
+            const float2 g2 = f2(G[i][2 * h], G[i][2 * h + 1]);
+            const float2 kn = __fmul2_rn(kv2, rk2), qn = __fmul2_rn(qv2, rq2);
+            const float2 da = __fadd2_rn(g2, f2(k4[CST_NREF][2 * h], k4[CST_NREF][2 * h + 1]));
+            const float2 db = __ffma2_rn(g2, m1, f2(k4[CST_GE][2 * h], k4[CST_GE][2 * h + 1]));
+            const float2 fA = f2(ex2(da.x), ex2(da.y));
+            const float2 kbe = __fmul2_rn(kn, f2(ex2(db.x), ex2(db.y)));
+            const float2 ka = __fmul2_rn(kn, fA), qa = __fmul2_rn(qn, fA);
+            const float2 p2r = f2(k4[CST_P2REF][2 * h], k4[CST_P2REF][2 * h + 1]);
+            const float2 kt = __fmul2_rn(ka, p2r), qt = __fmul2_rn(qa, p2r);
+            const float2 kh = __fmul2_rn(kbe, f2(k4[CST_KFAC][2 * h], k4[CST_KFAC][2 * h + 1]));
+            const float2 b0 = __fmul2_rn(kbe, f2(k4[CST_CDIAG][2 * h], k4[CST_CDIAG][2 * h + 1]));
+            const float2 b2 = __fmul2_rn(kbe, f2(k4[CST_C2][2 * h], k4[CST_C2][2 * h + 1]));
+            const float2 b3 = __fmul2_rn(kbe, f2(k4[CST_C3][2 * h], k4[CST_C3][2 * h + 1]));
+            pa[h] = pack_bf16(ka.x, ka.y);
+            pq[h] = pack_bf16(qa.x, qa.y);
+            pqt[h] = pack_bf16(qt.x, qt.y);
+            pkt[h] = pack_bf16(kt.x, kt.y);
+            pkh[h] = pack_bf16(kh.x, kh.y);
+            const float2 rem = __fadd2_rn(kh, f2(-bf16_lo_of(pkh[h]), -bf16_hi_of(pkh[h])));
+            pkl[h] = pack_bf16(rem.x, rem.y);
+            pb0[h] = pack_bf16(b0.x, b0.y);
+            pb1[h] = pack_bf16(kbe.x, kbe.y);  // B^(Jb+1): reference row is this block's last row
+            pb2[h] = pack_bf16(b2.x, b2.y);
+            pb3[h] = pack_bf16(b3.x, b3.y);
           }
-        };
-        switch (Jb) {
-          case 0: rows(std::integral_constant<int, 0>{}); break;
-          case 1: rows(std::integral_constant<int, 1>{}); break;
-          case 2: rows(std::integral_constant<int, 2>{}); break;
-          default: rows(std::integral_constant<int, 3>{}); break;
+          khlo[i] = make_uint2(pkl[0], pkl[1]);
+          uint8_t* aop = sm + SM_AOP + colhalf * 16384u + io[i];
+          uint8_t* bst = sm + SM_BT + colhalf * (BT_ROWS * 128u) + io[i];
+          *reinterpret_cast<uint2*>(aop) = make_uint2(pa[0], pa[1]);
+          *reinterpret_cast<uint2*>(aop + 8192) = make_uint2(pq[0], pq[1]);
+          *reinterpret_cast<uint2*>(sq + OFF_Q + colhalf * QGV_ATOM + io[i]) = make_uint2(pqt[0], pqt[1]);
+          *reinterpret_cast<uint2*>(sq + OFF_K + colhalf * K_ATOM + io[i]) = make_uint2(pkh[0], pkh[1]);
+          *reinterpret_cast<uint2*>(sq + OFF_G + colhalf * QGV_ATOM + io[i]) = make_uint2(pkt[0], pkt[1]);
+          *reinterpret_cast<uint2*>(bst + dcol(Jb) * 128u) = make_uint2(pb0[0], pb0[1]);  // diagonal
+          if (Jb + 1 <= 3)
+            *reinterpret_cast<uint2*>(bst + dcol(Jb + 1) * 128u) = make_uint2(pb1[0], pb1[1]);
+          if (Jb + 2 <= 3)
+            *reinterpret_cast<uint2*>(bst + dcol(Jb + 2) * 128u) = make_uint2(pb2[0], pb2[1]);
+          if (Jb + 3 <= 3)
+            *reinterpret_cast<uint2*>(bst + dcol(Jb + 3) * 128u) = make_uint2(pb3[0], pb3[1]);
+          if (!valid || it.zero_v)  // an M run treats v as zero
+            *reinterpret_cast<uint2*>(sq + OFF_V + colhalf * QGV_ATOM + io[i]) = make_uint2(0, 0);
         }
       }
       if (st_thread) tma_store_wait_read();  // the previous out tile (in the K^ lo region) was read
@@ -840,25 +911,107 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 
       // =================== phase 3: T, Aqk, solve ===================
-      // fp32 scratch in the B-tile region (free once the intra MMA has completed)
-      constexpr int TP = 68, YP = 36;                       // row pitches (floats)
+      // X = (I + T)^-1 by 16x16 blocks: the four diagonal inverses P_I = (I + T_II)^-1 by
+      // forward substitution in registers, then every off-diagonal block by block forward
+      // substitution, X_IJ = -P_I sum_{J<=K<I} T_IK X_KJ, rearranged into rounds of independent
+      // 16x16 products (one per warp pair) so that the chain is four products long:
+      //   R2: A_IJ = T_IJ P_J (six),  G21 = -P2 T21,  G31 = -P3 T31
+      //   R3: X10 = -P1 A10, X21 = -P2 A21, X32 = -P3 A32, D_IJ = -P_I A_IJ (IJ = 20, 31, 30),
+      //       G32 = -P3 T32
+      //   R4: X20 = D20 + G21 X10,  X31 = D31 + G32 X21,  E30 = D30 + G31 X10
+      //   R5: X30 = E30 + G32 X20
+      // Each finished block goes straight out as Xsol = X diag(beta) in bf16 hi and lo parts.
+      constexpr int TP = kSolveTP;
       float* Ts = reinterpret_cast<float*>(sm + SM_BT);   // T = stril(diag(beta) K~ K-^T) [64][TP]
-      float* Xs = Ts + 64 * TP;                           // X = (I + T)^-1            [64][TP]
-      float* Ys = Xs + 64 * TP;                           // block products            [32][YP]
+      float* Xs = Ts + 64 * TP;                           // X = (I + T)^-1 (lower blocks) [64][TP]
+      auto XB = [&](int I, int J) { return Xs + 16 * I * TP + 16 * J; };
+      // Xsol row 16 I + i, columns 16 J + j .. + 3 (bf16 hi in rows 0-63, lo in rows 64-127)
+      auto put_xsol = [&](int I, int J, int i, int j, float x0, float x1, float x2, float x3) {
+        const float4 b4 = *reinterpret_cast<const float4*>(beta_s + 16 * J + j);
+        const float f0 = x0 * b4.x, f1 = x1 * b4.y, f2 = x2 * b4.z, f3 = x3 * b4.w;
+        const uint2 hi = pack4(f0, f1, f2, f3);
+        const uint2 lo = make_uint2(split_lo(f0, f1, hi.x), split_lo(f2, f3, hi.y));
+        *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 16 * I + i, 16 * J + j)) = hi;
+        *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 64 + 16 * I + i, 16 * J + j)) = lo;
+      };
+      // O = C + sg (L R) for 16x16 fp32 blocks by one warp on the warp-level tensor-core path
+      // (mma.sync m16n8k8, tf32; two 8-column halves).  Each operand is split into a tf32 high
+      // part and a tf32 remainder and multiplied as hi*hi + hi*lo + lo*hi, which keeps about the
+      // precision of fp32 products.  With xI >= 0, O is the final block X_(xI,xJ) and also goes
+      // out as Xsol.
+      auto bprod = [&](const float* L, int ldl, const float* R, int ldr, const float* C, int ldc,
+                       float sg, float* O, int ldo, int xI, int xJ) {
+        const int g = lane >> 2, t = lane & 3;
+        float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float av[2][4], bv[2][2][2];
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const int k0 = 8 * kk + t;
+          av[kk][0] = L[g * ldl + k0];
+          av[kk][1] = L[(g + 8) * ldl + k0];
+          av[kk][2] = L[g * ldl + k0 + 4];
+          av[kk][3] = L[(g + 8) * ldl + k0 + 4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            bv[kk][h][0] = R[k0 * ldr + 8 * h + g];
+            bv[kk][h][1] = R[(k0 + 4) * ldr + 8 * h + g];
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          uint32_t ah[4], al[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            ah[e] = to_tf32(av[kk][e]);
+            al[e] = to_tf32(av[kk][e] - __uint_as_float(ah[e]));
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t bh[2], bl[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              bh[e] = to_tf32(bv[kk][h][e]);
+              bl[e] = to_tf32(bv[kk][h][e] - __uint_as_float(bh[e]));
+            }
+            mma_tf32_m16n8k8(d[h], al, bh);
+            mma_tf32_m16n8k8(d[h], ah, bl);
+            mma_tf32_m16n8k8(d[h], ah, bh);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c0 = 8 * h + 2 * t;
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const int i = g + 8 * hr;
+            float2 cv = make_float2(0.f, 0.f);
+            if (C) cv = *reinterpret_cast<const float2*>(C + i * ldc + c0);
+            const float o0 = fmaf(sg, d[h][2 * hr], cv.x), o1 = fmaf(sg, d[h][2 * hr + 1], cv.y);
+            *reinterpret_cast<float2*>(O + i * ldo + c0) = make_float2(o0, o1);
+            if (xI >= 0) {
+              const float2 b2 = *reinterpret_cast<const float2*>(beta_s + 16 * xJ + c0);
+              const float f0 = o0 * b2.x, f1 = o1 * b2.y;
+              const uint32_t hi = pack_bf16(f0, f1);
+              *reinterpret_cast<uint32_t*>(sm + SM_XSOL + sw128_offset(128, 16 * xI + i, 16 * xJ + c0)) = hi;
+              *reinterpret_cast<uint32_t*>(sm + SM_XSOL + sw128_offset(128, 64 + 16 * xI + i, 16 * xJ + c0)) =
+                  split_lo(f0, f1, hi);
+            }
+          }
+        }
+      };
       {
         // TMEM lane quarter q4 = warp & 3 holds rows 32 (q4 & 1) .. +31 of k (q4 < 2) or q (q4 >= 2),
         // i.e. row blocks bA = 2 (q4 & 1) and bA + 1.  Items are (block, 16-column chunk); chunks
         // right of a block's diagonal are zero.  q rows (Aqk): the quarter's 8 items, 2 a warp.
-        // k rows (T), default solve: warps 0 and 1 take the four diagonal 16x16 blocks, all that
-        // the first solve level reads, and start it at once; warps 4, 5, 9, 13 take the six
-        // off-diagonal blocks meanwhile.
+        // k rows (T): warps 0 and 1 take the four diagonal 16x16 blocks, all that the first solve
+        // round reads, and start it at once; warps 4, 5, 9, 13 take the six off-diagonal blocks
+        // meanwhile.
         const int q4 = warp & 3;
         const int r = (q4 & 1) * 32 + lane;
         const bool krow = q4 < 2;
         const float br = krow ? beta_s[r] : 0.f;
         const int bA = 2 * (q4 & 1);
         auto item_at = [&](int it, int& blk, int& ch) -> bool {
-#if KDA_SOLVE_L1 == 0
           if (krow) {
             if (wg == 0) {  // warp 0: (0,0) (1,1); warp 1: (2,2) (3,3)
               blk = ch = bA + it;
@@ -875,7 +1028,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ch = (k < 2) ? k : k - 2;
             return k < 5;
           }
-#endif
           const int item = 2 * wg + it;
           blk = bA + (item >> 2);
           ch = item & 3;
@@ -923,337 +1075,70 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (has0) put(blk0, ch0, va);
           if (has1) put(blk1, ch1, vb);
         }
-        // the merges read strictly upper blocks of X that no level writes: X(0:16, 16:32) and
-        // X(32:48, 48:64) (16x16), and the upper 8x8 block of each 16x16 diagonal block
-        // (threads 64-255: warps 0 and 1 go on to the first level)
-        const int zt = tid - 64;
-        if (zt >= 0 && zt < 128) {
-          const int blk2 = zt >> 6, rr = (zt & 63) >> 2, c4 = (zt & 3) * 4;
-          *reinterpret_cast<float4*>(Xs + (32 * blk2 + rr) * TP + 32 * blk2 + 16 + c4) =
-              make_float4(0.f, 0.f, 0.f, 0.f);
-        } else if (zt >= 128 && zt < 192) {
-          const int I = (zt - 128) >> 4, rr = ((zt - 128) >> 1) & 7, c4 = (zt & 1) * 4;
-          *reinterpret_cast<float4*>(Xs + (16 * I + rr) * TP + 16 * I + 8 + c4) =
-              make_float4(0.f, 0.f, 0.f, 0.f);
+        // warps 8 and 12 extract nothing: they zero Xsol's blocks above the diagonal meanwhile
+        if (warp == 8 || warp == 12) {
+          const int t = (warp >> 2) * 32 - 64 + lane;  // 0..63
+#pragma unroll 1
+          for (int e = t; e < 6 * 16 * 4; e += 64) {
+            const int blkp = e >> 6, i = (e >> 2) & 15, j = 4 * (e & 3);
+            // upper blocks (I, J), J > I: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+            const int I = (blkp < 3) ? 0 : (blkp < 5) ? 1 : 2;
+            const int J = (blkp < 3) ? blkp + 1 : (blkp < 5) ? blkp - 1 : 3;
+            *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 16 * I + i, 16 * J + j)) =
+                make_uint2(0u, 0u);
+            *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 64 + 16 * I + i, 16 * J + j)) =
+                make_uint2(0u, 0u);
+          }
         }
       }
-#if KDA_SOLVE_L1 == 0
-      // level 1 (default) while the other warps finish the extraction: the 8x8 diagonal
-      // inverses on warps 0 and 1, then the 8->16 merges on warps 0, 1, 8 and 12 (warps 8 and 12
-      // extract nothing); barriers among those warps only
-      const bool l1_warp = warp < 2 || warp == 8 || warp == 12;
+      // R1 (warps 0 and 1, while the others finish the extraction): P_I = (I + T_II)^-1; lane
+      // (I, c) computes column c by forward substitution over the rows of block I
       if (warp < 2) {
         named_bar_sync(1, 64);  // both warps' diagonal blocks of T are in Ts
-        {
-          // level 1a: X_mm = (I + T_mm)^-1 for the eight 8x8 diagonal blocks; thread = (block,
-          // column), rows by forward substitution as dot products over the final entries
-          const int base = 8 * (tid >> 3), cc = tid & 7;
-          float x[8];
-          x[0] = (cc == 0) ? 1.f : 0.f;
-#pragma unroll
-          for (int rr = 1; rr < 8; ++rr) {
-            const float* trow = Ts + (base + rr) * TP + base;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < rr; k0 += 4) {
-              const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
-              const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
-            }
-            const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-            x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k) Xs[(base + k) * TP + base + cc] = x[k];
-        }
-      }
-      if (l1_warp) {
-        named_bar_sync(2, 128);  // the 8x8 inverses are in Xs
-        // level 1b: X_(16I+8.., 16I..) = -X22 T21 X11 inside each 16x16 diagonal block; thread =
-        // (row rr, column cc) of blocks I0 and I0 + 1
-        const int t128 = (warp < 2 ? warp : (warp >> 2)) * 32 + lane;  // warps 0, 1, 8, 12 -> 0..127
-        const int rr = (t128 >> 3) & 7, cc = t128 & 7, I0 = 2 * (t128 >> 6);
-#pragma unroll
-        for (int I = I0; I < I0 + 2; ++I) {
-          const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
-          const float4 ta = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1);
-          const float4 tb = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1 + 4);
-          const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-          float y = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) y = fmaf(tv[k], Xs[(c1 + k) * TP + c1 + cc], y);
-          Ys[(8 * I + rr) * YP + cc] = y;
-        }
-        named_bar_sync(2, 128);
-#pragma unroll
-        for (int I = I0; I < I0 + 2; ++I) {
-          const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
-          const float4 xa = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 8);
-          const float4 xb = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 12);
-          const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-          float z = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) z = fmaf(xv[k], Ys[(8 * I + k) * YP + cc], z);
-          Xs[r1 * TP + c1 + cc] = -z;
-        }
-      }
-      __syncthreads();
-      KDA_TS(13);
-      KDA_TS(14);
-#else
-      __syncthreads();
-      KDA_TS(13);
-#endif
-#if KDA_SOLVE_L1 == 1
-      // level 1 (variant 1): the 16x16 diagonal inverses by column forward substitution, one
-      // thread per (block, column); two merge levels follow
-      if (tid < 64) {
-        const int I = tid >> 4, cc = tid & 15, base = 16 * I;
+        const int I = 2 * warp + (lane >> 4), c = lane & 15, base = 16 * I;
         float x[16];
-        x[0] = (cc == 0) ? 1.f : 0.f;
+        x[0] = (c == 0) ? 1.f : 0.f;
 #pragma unroll
-        for (int rr = 1; rr < 16; ++rr) {
-          const float* trow = Ts + (base + rr) * TP + base;
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int r = 1; r < 16; ++r) {
+          const float* trow = Ts + (base + r) * TP + base;
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-          for (int k0 = 0; k0 < rr; k0 += 4) {
-            const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
-            const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
+          for (int s0 = 0; s0 < r; s0 += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(trow + s0);
+            if (s0 + 0 < r) a0 = fmaf(t4.x, x[s0 + 0], a0);
+            if (s0 + 1 < r) a1 = fmaf(t4.y, x[s0 + 1], a1);
+            if (s0 + 2 < r) a0 = fmaf(t4.z, x[s0 + 2], a0);
+            if (s0 + 3 < r) a1 = fmaf(t4.w, x[s0 + 3], a1);
           }
-          const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-          x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
+          x[r] = (r == c) ? 1.f : -(a0 + a1);
         }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) Xs[(base + k) * TP + base + cc] = x[k];
+        for (int r = 0; r < 16; ++r) Xs[(base + r) * TP + base + c] = x[r];
       }
       __syncthreads();
-      KDA_TS(14);
-#elif KDA_SOLVE_L1 == 2
-      // level 1 (variant 2): 8x8 inverses and their 8->16 merge warp-local, one warp per 16x16
-      // block (warps 0, 4, 8, 12), synchronised within the warp only
-      if ((warp & 3) == 0) {
-        const int I = wg;
-        if (lane < 16) {
-          const int base = 16 * I + 8 * (lane >> 3), cc = lane & 7;
-          float x[8];
-          x[0] = (cc == 0) ? 1.f : 0.f;
-#pragma unroll
-          for (int rr = 1; rr < 8; ++rr) {
-            const float* trow = Ts + (base + rr) * TP + base;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < rr; k0 += 4) {
-              const float4 t4 = *reinterpret_cast<const float4*>(trow + k0);
-              const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (k0 + e < rr) acc[e] = fmaf(tv[e], x[k0 + e], acc[e]);
-            }
-            const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-            x[rr] = (rr == cc) ? 1.f : ((rr < cc) ? 0.f : -sum);
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k) Xs[(base + k) * TP + base + cc] = x[k];
-        }
-        __syncwarp();
-        const int rr = lane >> 2, cb = (lane & 3) * 2;
-        const int r1 = 16 * I + 8 + rr, c1 = 16 * I;
-        {
-          const float4 ta = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1);
-          const float4 tb = *reinterpret_cast<const float4*>(Ts + r1 * TP + c1 + 4);
-          const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-          float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float2 xv = *reinterpret_cast<const float2*>(Xs + (c1 + k) * TP + c1 + cb);
-            y0 = fmaf(tv[k], xv.x, y0);
-            y1 = fmaf(tv[k], xv.y, y1);
-          }
-          *reinterpret_cast<float2*>(Ys + (8 * I + rr) * YP + cb) = make_float2(y0, y1);
-        }
-        __syncwarp();
-        {
-          const float4 xa = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 8);
-          const float4 xb = *reinterpret_cast<const float4*>(Xs + r1 * TP + c1 + 12);
-          const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-          float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float2 yv = *reinterpret_cast<const float2*>(Ys + (8 * I + k) * YP + cb);
-            z0 = fmaf(xv[k], yv.x, z0);
-            z1 = fmaf(xv[k], yv.y, z1);
-          }
-          *reinterpret_cast<float2*>(Xs + r1 * TP + c1 + cb) = make_float2(-z0, -z1);
-        }
-      }
-      __syncthreads();
-      KDA_TS(14);
-#endif
-      // level 2: X_{I,I-1} = -X_II T_{I,I-1} X_{I-1,I-1} for I = 1, 3 (two 16x16 merges).  A thread
-      // owns a 2x2 output tile and a quarter of the inner dimension; the quarters meet by shuffles.
-      {
-        const int kq = lane & 3, tile = warp * 8 + (lane >> 2);
-        const int pI = tile >> 6, tr = (tile >> 3) & 7, tc = tile & 7;
-        const int I = 2 * pI + 1, J = I - 1;
-        const int ra = 16 * I + 2 * tr, cb = 2 * tc;
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-        {
-          const float4 ta = *reinterpret_cast<const float4*>(Ts + ra * TP + 16 * J + 4 * kq);
-          const float4 tb = *reinterpret_cast<const float4*>(Ts + (ra + 1) * TP + 16 * J + 4 * kq);
-          const float tav[4] = {ta.x, ta.y, ta.z, ta.w}, tbv[4] = {tb.x, tb.y, tb.z, tb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 xv = *reinterpret_cast<const float2*>(Xs + (16 * J + 4 * kq + e) * TP + 16 * J + cb);
-            y00 = fmaf(tav[e], xv.x, y00);
-            y01 = fmaf(tav[e], xv.y, y01);
-            y10 = fmaf(tbv[e], xv.x, y10);
-            y11 = fmaf(tbv[e], xv.y, y11);
-          }
-        }
-#pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-          y00 += __shfl_xor_sync(0xffffffffu, y00, o);
-          y01 += __shfl_xor_sync(0xffffffffu, y01, o);
-          y10 += __shfl_xor_sync(0xffffffffu, y10, o);
-          y11 += __shfl_xor_sync(0xffffffffu, y11, o);
-        }
-        if (kq == 0) {
-          *reinterpret_cast<float2*>(Ys + (16 * pI + 2 * tr) * YP + cb) = make_float2(y00, y01);
-          *reinterpret_cast<float2*>(Ys + (16 * pI + 2 * tr + 1) * YP + cb) = make_float2(y10, y11);
-        }
-        __syncthreads();
-        float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
-        {
-          const float4 xa = *reinterpret_cast<const float4*>(Xs + ra * TP + 16 * I + 4 * kq);
-          const float4 xb = *reinterpret_cast<const float4*>(Xs + (ra + 1) * TP + 16 * I + 4 * kq);
-          const float xav[4] = {xa.x, xa.y, xa.z, xa.w}, xbv[4] = {xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 yv = *reinterpret_cast<const float2*>(Ys + (16 * pI + 4 * kq + e) * YP + cb);
-            z00 = fmaf(xav[e], yv.x, z00);
-            z01 = fmaf(xav[e], yv.y, z01);
-            z10 = fmaf(xbv[e], yv.x, z10);
-            z11 = fmaf(xbv[e], yv.y, z11);
-          }
-        }
-#pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-          z00 += __shfl_xor_sync(0xffffffffu, z00, o);
-          z01 += __shfl_xor_sync(0xffffffffu, z01, o);
-          z10 += __shfl_xor_sync(0xffffffffu, z10, o);
-          z11 += __shfl_xor_sync(0xffffffffu, z11, o);
-        }
-        if (kq == 0) {
-          *reinterpret_cast<float2*>(Xs + ra * TP + 16 * J + cb) = make_float2(-z00, -z01);
-          *reinterpret_cast<float2*>(Xs + (ra + 1) * TP + 16 * J + cb) = make_float2(-z10, -z11);
-        }
-      }
-      __syncthreads();
-      KDA_TS(15);
-      // level 3: X_(32:64, 0:32) = -X_(32:64, 32:64) T_(32:64, 0:32) X_(0:32, 0:32) (32x32 merge).
-      // A thread owns a 4x2 output tile and the inner indices 4 kq + e + 16 m (e < 4, m < 2): the
-      // four kq of a warp read rows 4 apart, two 16-bank halves, so each load is 2 wavefronts.
-      {
-        const int kq = lane & 3, tile = warp * 8 + (lane >> 2);
-        const int ra = 32 + 4 * (tile >> 4), cb = 2 * (tile & 15);
-        // X_(0:32, 0:32) is zero in rows 0-15 of columns 16-31, so tiles right of column 16 (odd
-        // warps) need only m = 1 here; X_(32:64, 32:64) is zero in columns 48-63 of rows 32-47,
-        // so rows below 48 (warps 0-7) need only m = 0 in the second product.
-        const int m_lo = (warp & 1) ? 1 : 0, m_hi = (warp < 8) ? 1 : 2;
-        float acc[4][2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
+      KDA_TS(13);
+      // R2 .. R5 on warps 0-7, one product per warp and round (barriers among those warps only);
+      // warps 8-15 write the diagonal blocks' Xsol meanwhile
+      if (warp < 8) {
 #pragma unroll 1
-        for (int m = m_lo; m < 2; ++m) {
-          const int kb = 4 * kq + 16 * m;
-          float tv[4][4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 t4 = *reinterpret_cast<const float4*>(Ts + (ra + i) * TP + kb);
-            tv[i][0] = t4.x; tv[i][1] = t4.y; tv[i][2] = t4.z; tv[i][3] = t4.w;
+        for (int rd = 0; rd < 4; ++rd) {
+          const SolveOp op = kSolveOps[rd][warp];
+          if (op.sg != 0) {
+            float* F = reinterpret_cast<float*>(sm);
+            bprod(F + op.l, op.ldl, F + op.r, op.ldr, op.c ? F + op.c : nullptr, op.ldc,
+                  (float)op.sg, F + op.o, op.ldo, op.xi, op.xj);
           }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 xv = *reinterpret_cast<const float2*>(Xs + (kb + e) * TP + cb);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              acc[i][0] = fmaf(tv[i][e], xv.x, acc[i][0]);
-              acc[i][1] = fmaf(tv[i][e], xv.y, acc[i][1]);
-            }
-          }
+          if (rd == 0) KDA_TS(22);
+          if (rd < 3) named_bar_sync(2, 256);
+          if (rd == 0) KDA_TS(14);
+          if (rd == 1) KDA_TS(15);
         }
-#pragma unroll
-        for (int o = 1; o < 4; o <<= 1)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[i][0] += __shfl_xor_sync(0xffffffffu, acc[i][0], o);
-            acc[i][1] += __shfl_xor_sync(0xffffffffu, acc[i][1], o);
-          }
-        if (kq == 0) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float2*>(Ys + (ra - 32 + i) * YP + cb) = make_float2(acc[i][0], acc[i][1]);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
-#pragma unroll 1
-        for (int m = 0; m < m_hi; ++m) {
-          const int kb = 4 * kq + 16 * m;
-          float xv4[4][4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 x4 = *reinterpret_cast<const float4*>(Xs + (ra + i) * TP + 32 + kb);
-            xv4[i][0] = x4.x; xv4[i][1] = x4.y; xv4[i][2] = x4.z; xv4[i][3] = x4.w;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 yv = *reinterpret_cast<const float2*>(Ys + (kb + e) * YP + cb);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              acc[i][0] = fmaf(xv4[i][e], yv.x, acc[i][0]);
-              acc[i][1] = fmaf(xv4[i][e], yv.y, acc[i][1]);
-            }
-          }
-        }
-#pragma unroll
-        for (int o = 1; o < 4; o <<= 1)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[i][0] += __shfl_xor_sync(0xffffffffu, acc[i][0], o);
-            acc[i][1] += __shfl_xor_sync(0xffffffffu, acc[i][1], o);
-          }
-        if (kq == 0) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float2*>(Xs + (ra + i) * TP + cb) = make_float2(-acc[i][0], -acc[i][1]);
-        }
+      } else {
+        const int t = tid - 256, I = t >> 6, i = (t >> 2) & 15, j = 4 * (t & 3);
+        const float4 x4 = *reinterpret_cast<const float4*>(XB(I, I) + i * TP + j);
+        put_xsol(I, I, i, j, x4.x, x4.y, x4.z, x4.w);
       }
-      __syncthreads();
       KDA_TS(16);
-      // Xsol = X diag(beta) -> bf16 hi (rows 0-63) and lo (rows 64-127) parts, K-major [r][s]
-      {
-        const int r = tid >> 3, s0 = (tid & 7) * 8;
-        const float4 xa = *reinterpret_cast<const float4*>(Xs + r * TP + s0);
-        const float4 xb = *reinterpret_cast<const float4*>(Xs + r * TP + s0 + 4);
-        const float4 ba = *reinterpret_cast<const float4*>(beta_s + s0);
-        const float4 bb = *reinterpret_cast<const float4*>(beta_s + s0 + 4);
-        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        const float bv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = (s0 + e <= r) ? xv[e] * bv[e] : 0.f;
-        const uint4 hi = pack8(f);
-        const uint4 lo = make_uint4(split_lo(f[0], f[1], hi.x), split_lo(f[2], f[3], hi.y),
-                                    split_lo(f[4], f[5], hi.z), split_lo(f[6], f[7], hi.w));
-        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, r, s0)) = hi;
-        *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, 64 + r, s0)) = lo;
-      }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();

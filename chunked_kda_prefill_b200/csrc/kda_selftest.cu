@@ -193,8 +193,25 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
+// y[i] = ex2(x[i]): the SFU exponential every decay of the fused kernel goes through.
+__global__ void ex2_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = ex2(x[i]);
+}
+
 }  // namespace
 }  // namespace kda
+
+// Internal entry point (not part of include/kda.h): y = ex2.approx.ftz.f32(x) elementwise on the
+// device, for a host-side accuracy check of the instruction.  Returns 0, 1 (bad argument) or 2.
+extern "C" __attribute__((visibility("default"))) int kda_selftest_ex2(const float* x, float* y,
+                                                                       int n, void* stream) {
+  if (!x || !y || n < 1) return 1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  kda::ex2_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y, n);
+  if (cudaGetLastError() != cudaSuccess) return 2;
+  return cudaStreamSynchronize(s) == cudaSuccess ? 0 : 2;
+}
 
 // Returns 0 on success, 1 on a bad argument, 2 on a CUDA error, 3 if a bounded wait gave up.
 extern "C" __attribute__((visibility("default"))) int kda_selftest(

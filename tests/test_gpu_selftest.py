@@ -124,3 +124,28 @@ def test_device_timeout_word_maps_to_status_code(cuda_ok):
         with pytest.raises(kda.KdaError) as e:
             kda.device_status(ws)
         assert e.value.name == name
+
+
+def test_ex2_accuracy(cuda_ok):
+    """ex2.approx.ftz.f32 (every decay factor 2^x of the fused kernel) against exp2 in fp64 over
+    the arguments the kernel forms: gate arguments and log2-space cumulative-sum differences."""
+    L = kda.load()
+    f = L.kda_selftest_ex2
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    g = torch.Generator().manual_seed(5)
+    x = torch.cat([torch.linspace(-126.0, 127.0, 1 << 20, dtype=torch.float32),
+                   (torch.rand(1 << 20, generator=g) * 253.0 - 126.0).to(torch.float32),
+                   torch.tensor([-130.0, -150.0, -500.0], dtype=torch.float32)])
+    xd = x.cuda()
+    yd = torch.empty_like(xd)
+    assert f(xd.data_ptr(), yd.data_ptr(), x.numel(), torch.cuda.current_stream().cuda_stream) == 0
+    xs = x.double().numpy()
+    y = yd.cpu().double().numpy()
+    ref = np.exp2(xs)
+    normal = xs >= -125.0
+    rel = np.abs(y[normal] - ref[normal]) / ref[normal]
+    assert rel.max() < 2.0 ** -21, rel.max()
+    # results below the smallest normal float are flushed to zero (ftz)
+    assert np.all(y[xs <= -127.0] <= 2.0 ** -126)
+    print(f"ex2.approx.ftz.f32: max relative error {rel.max():.3e} = 2^{np.log2(rel.max()):.2f}")
