@@ -12,9 +12,9 @@
 //   2 MMA  D_I = Aop B^(I)^T, I = 0..3 (M=128, N=160 for all four blocks, K=128): rows 0-63 give
 //     T = stril(diag(beta) K~ K-^T), rows 64-127 give Aqk = tril(Q~ K-^T); meanwhile K^ lo is
 //     stored and the state left by the previous chunk becomes the bf16 hi/lo state operand
-//   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 16x16 blocks (diagonal inverses in registers,
-//     then rounds of independent block products); Xsol = X diag(beta) -> bf16 hi and lo parts
-//     stacked as one 128-row operand
+//   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 32x32 blocks (diagonal inverses by forward
+//     substitution in registers, then the off-diagonal block by two block products);
+//     Xsol = X diag(beta) -> bf16 hi and lo parts stacked as one 128-row operand
 //   4 MMA  W^T = K~^T [Xsol_hi; Xsol_lo]^T and U^T = V^T [Xsol_hi; Xsol_lo]^T (one N=128 chain
 //          each, hi and lo parts side by side); S <- S Diag(2^G_last)
 //     meanwhile.  Then -W -> bf16 hi and lo, stored token-major over the K~ and V tiles
@@ -123,53 +123,6 @@ enum : int { CST_NREF = 0, CST_GE, CST_P2REF, CST_KFAC, CST_CDIAG, CST_C2, CST_C
   } while (0)
 #endif
 
-// The triangular solve's rounds of 16x16 block products (phase 3): O = C + sg (L R), operands
-// as float offsets from the shared-memory base.  T and X are [64][kSolveTP] fp32 in the B-tile
-// region (free after the intra MMA), twelve scratch blocks Z0..Z11 [16][kSolveBP] in the upper
-// half of the Aop region; xi >= 0 marks a final block X_(xi,xj), also written out as Xsol.
-constexpr int kSolveTP = 68, kSolveBP = 20;
-struct SolveOp {
-  uint16_t l, ldl, r, ldr, c, ldc, o, ldo;  // offsets (floats) and row pitches
-  int8_t sg;                                 // sg == 0: no product;  c == 0: no C term
-  int8_t xi, xj, pad;
-};
-constexpr int kTs = (int)(SM_BT / 4), kXs = kTs + 64 * kSolveTP, kZs = (int)((SM_AOP + 16384) / 4);
-static_assert(kXs + 64 * kSolveTP <= (int)(SM_KLO / 4), "T and X overflow the B-tile region");
-static_assert(12 * 16 * kSolveBP <= 16384 / 4, "scratch blocks overflow the Aop upper half");
-static_assert(kZs + 12 * 16 * kSolveBP < 65536, "offsets must fit 16 bits");
-constexpr uint16_t TBo(int I, int J) { return (uint16_t)(kTs + 16 * I * kSolveTP + 16 * J); }
-constexpr uint16_t XBo(int I, int J) { return (uint16_t)(kXs + 16 * I * kSolveTP + 16 * J); }
-constexpr uint16_t ZBo(int z) { return (uint16_t)(kZs + z * 16 * kSolveBP); }
-constexpr uint16_t TPs = kSolveTP, BPs = kSolveBP;
-constexpr SolveOp kNoOp = {0, 0, 0, 0, 0, 0, 0, 0, 0, -1, 0, 0};
-__constant__ SolveOp kSolveOps[4][8] = {
-    {// R2: A_IJ = T_IJ P_J -> Z0..Z5;  G21 = -P2 T21 -> Z6;  G31 = -P3 T31 -> Z7
-     {TBo(1, 0), TPs, XBo(0, 0), TPs, 0, 0, ZBo(0), BPs, 1, -1, 0, 0},
-     {TBo(2, 1), TPs, XBo(1, 1), TPs, 0, 0, ZBo(1), BPs, 1, -1, 0, 0},
-     {TBo(3, 2), TPs, XBo(2, 2), TPs, 0, 0, ZBo(2), BPs, 1, -1, 0, 0},
-     {TBo(2, 0), TPs, XBo(0, 0), TPs, 0, 0, ZBo(3), BPs, 1, -1, 0, 0},
-     {TBo(3, 1), TPs, XBo(1, 1), TPs, 0, 0, ZBo(4), BPs, 1, -1, 0, 0},
-     {TBo(3, 0), TPs, XBo(0, 0), TPs, 0, 0, ZBo(5), BPs, 1, -1, 0, 0},
-     {XBo(2, 2), TPs, TBo(2, 1), TPs, 0, 0, ZBo(6), BPs, -1, -1, 0, 0},
-     {XBo(3, 3), TPs, TBo(3, 1), TPs, 0, 0, ZBo(7), BPs, -1, -1, 0, 0}},
-    {// R3: X10, X21, X32 = -P_I A_IJ;  D20, D31, D30 = -P_I A_IJ -> Z8..Z10;  G32 -> Z11
-     {XBo(1, 1), TPs, ZBo(0), BPs, 0, 0, XBo(1, 0), TPs, -1, 1, 0, 0},
-     {XBo(2, 2), TPs, ZBo(1), BPs, 0, 0, XBo(2, 1), TPs, -1, 2, 1, 0},
-     {XBo(3, 3), TPs, ZBo(2), BPs, 0, 0, XBo(3, 2), TPs, -1, 3, 2, 0},
-     {XBo(2, 2), TPs, ZBo(3), BPs, 0, 0, ZBo(8), BPs, -1, -1, 0, 0},
-     {XBo(3, 3), TPs, ZBo(4), BPs, 0, 0, ZBo(9), BPs, -1, -1, 0, 0},
-     {XBo(3, 3), TPs, ZBo(5), BPs, 0, 0, ZBo(10), BPs, -1, -1, 0, 0},
-     {XBo(3, 3), TPs, TBo(3, 2), TPs, 0, 0, ZBo(11), BPs, -1, -1, 0, 0},
-     kNoOp},
-    {// R4: X20 = D20 + G21 X10;  X31 = D31 + G32 X21;  E30 = D30 + G31 X10 -> Z0
-     {ZBo(6), BPs, XBo(1, 0), TPs, ZBo(8), BPs, XBo(2, 0), TPs, 1, 2, 0, 0},
-     {ZBo(11), BPs, XBo(2, 1), TPs, ZBo(9), BPs, XBo(3, 1), TPs, 1, 3, 1, 0},
-     {ZBo(7), BPs, XBo(1, 0), TPs, ZBo(10), BPs, ZBo(0), BPs, 1, -1, 0, 0},
-     kNoOp, kNoOp, kNoOp, kNoOp, kNoOp},
-    {// R5: X30 = E30 + G32 X20
-     {ZBo(11), BPs, XBo(2, 0), TPs, ZBo(0), BPs, XBo(3, 0), TPs, 1, 3, 0, 0},
-     kNoOp, kNoOp, kNoOp, kNoOp, kNoOp, kNoOp, kNoOp}};
-
 __device__ __forceinline__ uint32_t dcol(int I) { return 8u * I * (I + 1); }
 
 // Byte offset of element (row, col) of a 64-row tile stored as two 64-column atoms `atom` bytes
@@ -202,24 +155,6 @@ __device__ __forceinline__ uint32_t split_lo(float a, float b, uint32_t hi) {
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
-}
-
-// fp32 -> tf32 (round to nearest, ties away; the low 13 mantissa bits cleared)
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-// d += a b for one 16x8x8 tile on the warp-level tensor-core path (tf32 inputs, fp32 d), with
-// the PTX fragment layouts: a = A(g, t), A(g+8, t), A(g, t+4), A(g+8, t+4); b = B(t, g), B(t+4, g);
-// d = D(g, 2t), D(g, 2t+1), D(g+8, 2t), D(g+8, 2t+1), where g = lane / 4 and t = lane % 4.
-__device__ __forceinline__ void mma_tf32_m16n8k8(float (&d)[4], const uint32_t (&a)[4],
-                                                 const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 struct Maps {
@@ -911,101 +846,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 
       // =================== phase 3: T, Aqk, solve ===================
-      // X = (I + T)^-1 by 16x16 blocks: the four diagonal inverses P_I = (I + T_II)^-1 by
-      // forward substitution in registers, then every off-diagonal block by block forward
-      // substitution, X_IJ = -P_I sum_{J<=K<I} T_IK X_KJ, rearranged into rounds of independent
-      // 16x16 products (one per warp pair) so that the chain is four products long:
-      //   R2: A_IJ = T_IJ P_J (six),  G21 = -P2 T21,  G31 = -P3 T31
-      //   R3: X10 = -P1 A10, X21 = -P2 A21, X32 = -P3 A32, D_IJ = -P_I A_IJ (IJ = 20, 31, 30),
-      //       G32 = -P3 T32
-      //   R4: X20 = D20 + G21 X10,  X31 = D31 + G32 X21,  E30 = D30 + G31 X10
-      //   R5: X30 = E30 + G32 X20
-      // Each finished block goes straight out as Xsol = X diag(beta) in bf16 hi and lo parts.
-      constexpr int TP = kSolveTP;
+      // X = (I + T)^-1 by 32x32 blocks, A = rows/columns 0-31 and B = 32-63:
+      //   X_AA = (I + T_AA)^-1 and X_BB = (I + T_BB)^-1, one warp each, as soon as that warp has its
+      //     rows of T: two 16x16 diagonal inverses by column forward substitution (a half-warp
+      //     each, lane c computing column c in registers) and the block below them,
+      //     X_10 = -P_1 (T_10 P_0), by two 16x16x16 products;
+      //   X_BA = -X_BB (T_BA X_AA), two 32x32x32 products on warps 0-7 (lane i owns row i, warp w
+      //     columns 4w .. 4w+3; the right-hand operand is read warp-uniformly, a broadcast);
+      // Xsol = X diag(beta) goes out in bf16 hi and lo parts, the diagonal blocks by warps 8-15
+      // while the products run.
+      constexpr int TP = 68;                              // row pitch of T and X (floats)
+      constexpr int YP = 36;                              // row pitch of Y (floats)
       float* Ts = reinterpret_cast<float*>(sm + SM_BT);   // T = stril(diag(beta) K~ K-^T) [64][TP]
-      float* Xs = Ts + 64 * TP;                           // X = (I + T)^-1 (lower blocks) [64][TP]
-      auto XB = [&](int I, int J) { return Xs + 16 * I * TP + 16 * J; };
-      // Xsol row 16 I + i, columns 16 J + j .. + 3 (bf16 hi in rows 0-63, lo in rows 64-127)
-      auto put_xsol = [&](int I, int J, int i, int j, float x0, float x1, float x2, float x3) {
-        const float4 b4 = *reinterpret_cast<const float4*>(beta_s + 16 * J + j);
-        const float f0 = x0 * b4.x, f1 = x1 * b4.y, f2 = x2 * b4.z, f3 = x3 * b4.w;
-        const uint2 hi = pack4(f0, f1, f2, f3);
-        const uint2 lo = make_uint2(split_lo(f0, f1, hi.x), split_lo(f2, f3, hi.y));
-        *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 16 * I + i, 16 * J + j)) = hi;
-        *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 64 + 16 * I + i, 16 * J + j)) = lo;
-      };
-      // O = C + sg (L R) for 16x16 fp32 blocks by one warp on the warp-level tensor-core path
-      // (mma.sync m16n8k8, tf32; two 8-column halves).  Each operand is split into a tf32 high
-      // part and a tf32 remainder and multiplied as hi*hi + hi*lo + lo*hi, which keeps about the
-      // precision of fp32 products.  With xI >= 0, O is the final block X_(xI,xJ) and also goes
-      // out as Xsol.
-      auto bprod = [&](const float* L, int ldl, const float* R, int ldr, const float* C, int ldc,
-                       float sg, float* O, int ldo, int xI, int xJ) {
-        const int g = lane >> 2, t = lane & 3;
-        float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        float av[2][4], bv[2][2][2];
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int k0 = 8 * kk + t;
-          av[kk][0] = L[g * ldl + k0];
-          av[kk][1] = L[(g + 8) * ldl + k0];
-          av[kk][2] = L[g * ldl + k0 + 4];
-          av[kk][3] = L[(g + 8) * ldl + k0 + 4];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            bv[kk][h][0] = R[k0 * ldr + 8 * h + g];
-            bv[kk][h][1] = R[(k0 + 4) * ldr + 8 * h + g];
-          }
-        }
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          uint32_t ah[4], al[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            ah[e] = to_tf32(av[kk][e]);
-            al[e] = to_tf32(av[kk][e] - __uint_as_float(ah[e]));
-          }
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t bh[2], bl[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              bh[e] = to_tf32(bv[kk][h][e]);
-              bl[e] = to_tf32(bv[kk][h][e] - __uint_as_float(bh[e]));
-            }
-            mma_tf32_m16n8k8(d[h], al, bh);
-            mma_tf32_m16n8k8(d[h], ah, bl);
-            mma_tf32_m16n8k8(d[h], ah, bh);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int c0 = 8 * h + 2 * t;
-#pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            const int i = g + 8 * hr;
-            float2 cv = make_float2(0.f, 0.f);
-            if (C) cv = *reinterpret_cast<const float2*>(C + i * ldc + c0);
-            const float o0 = fmaf(sg, d[h][2 * hr], cv.x), o1 = fmaf(sg, d[h][2 * hr + 1], cv.y);
-            *reinterpret_cast<float2*>(O + i * ldo + c0) = make_float2(o0, o1);
-            if (xI >= 0) {
-              const float2 b2 = *reinterpret_cast<const float2*>(beta_s + 16 * xJ + c0);
-              const float f0 = o0 * b2.x, f1 = o1 * b2.y;
-              const uint32_t hi = pack_bf16(f0, f1);
-              *reinterpret_cast<uint32_t*>(sm + SM_XSOL + sw128_offset(128, 16 * xI + i, 16 * xJ + c0)) = hi;
-              *reinterpret_cast<uint32_t*>(sm + SM_XSOL + sw128_offset(128, 64 + 16 * xI + i, 16 * xJ + c0)) =
-                  split_lo(f0, f1, hi);
-            }
-          }
-        }
-      };
+      float* Xs = Ts + 64 * TP;                           // X_AA and X_BB               [64][TP]
+      float* Ys = reinterpret_cast<float*>(sm + SM_AOP + 16384);  // Y = T_BA X_AA     [32][YP]
+      // (Xs ends inside the B-tile region; Ys lies in Aop's upper half, free after the intra MMA)
       {
         // TMEM lane quarter q4 = warp & 3 holds rows 32 (q4 & 1) .. +31 of k (q4 < 2) or q (q4 >= 2),
-        // i.e. row blocks bA = 2 (q4 & 1) and bA + 1.  Items are (block, 16-column chunk); chunks
-        // right of a block's diagonal are zero.  q rows (Aqk): the quarter's 8 items, 2 a warp.
-        // k rows (T): warps 0 and 1 take the four diagonal 16x16 blocks, all that the first solve
-        // round reads, and start it at once; warps 4, 5, 9, 13 take the six off-diagonal blocks
-        // meanwhile.
+        // i.e. row blocks bA = 2 (q4 & 1) and bA + 1.  Items are (16-row block, 16-column chunk);
+        // chunks right of a block's diagonal are zero.  q rows (Aqk): the quarter's 8 items, 2 a
+        // warp.  k rows (T): warp 0 takes T_AA's three chunks (0,0) (1,0) (1,1) and warp 1 T_BB's
+        // (2,2) (3,2) (3,3), so each can start its diagonal inverse at once; warps 5 and 9 take T_BA.
         const int q4 = warp & 3;
         const int r = (q4 & 1) * 32 + lane;
         const bool krow = q4 < 2;
@@ -1013,25 +874,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bA = 2 * (q4 & 1);
         auto item_at = [&](int it, int& blk, int& ch) -> bool {
           if (krow) {
-            if (wg == 0) {  // warp 0: (0,0) (1,1); warp 1: (2,2) (3,3)
-              blk = ch = bA + it;
+            if (wg == 0) {
+              blk = bA + (it > 0 ? 1 : 0);
+              ch = bA + (it == 2 ? 1 : 0);
               return true;
             }
-            if (q4 == 0) {  // block row 1 has one off-diagonal chunk: warp 4
-              blk = 1;
-              ch = 0;
-              return wg == 1 && it == 0;
-            }
-            // (2,0) (2,1) | (3,0) (3,1) | (3,2) on warps 5, 9, 13
-            const int k = 2 * (wg - 1) + it;
-            blk = (k < 2) ? 2 : 3;
-            ch = (k < 2) ? k : k - 2;
-            return k < 5;
+            blk = 2 + (it & 1);  // warp 5: (2,0) (3,0); warp 9: (2,1) (3,1)
+            ch = wg - 1;
+            return q4 == 1 && (wg == 1 || wg == 2) && it < 2;
           }
           const int item = 2 * wg + it;
           blk = bA + (item >> 2);
           ch = item & 3;
-          return true;
+          return it < 2;
         };
         // an item's 16 columns of its block's rows -> T (fp32, scaled by beta) or Aqk (bf16),
         // strictly lower / lower parts; chunks right of the diagonal of an Aqk block are zeroed
@@ -1064,79 +919,142 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
         {
-          // both items' TMEM loads in one round trip
-          int blk0, ch0, blk1, ch1;
-          const bool has0 = item_at(0, blk0, ch0), has1 = item_at(1, blk1, ch1);
-          uint32_t va[16], vb[16];
-          // (unconditional loads: an item without data reads its block's first chunk, unused)
-          tmem_ld16(tl + TC_D + dcol(blk0) + 16 * ((has0 && ch0 <= blk0) ? ch0 : 0), va);
-          tmem_ld16(tl + TC_D + dcol(blk1) + 16 * ((has1 && ch1 <= blk1) ? ch1 : 0), vb);
-          tmem_wait_ld();
-          if (has0) put(blk0, ch0, va);
-          if (has1) put(blk1, ch1, vb);
-        }
-        // warps 8 and 12 extract nothing: they zero Xsol's blocks above the diagonal meanwhile
-        if (warp == 8 || warp == 12) {
-          const int t = (warp >> 2) * 32 - 64 + lane;  // 0..63
-#pragma unroll 1
-          for (int e = t; e < 6 * 16 * 4; e += 64) {
-            const int blkp = e >> 6, i = (e >> 2) & 15, j = 4 * (e & 3);
-            // upper blocks (I, J), J > I: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-            const int I = (blkp < 3) ? 0 : (blkp < 5) ? 1 : 2;
-            const int J = (blkp < 3) ? blkp + 1 : (blkp < 5) ? blkp - 1 : 3;
-            *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 16 * I + i, 16 * J + j)) =
-                make_uint2(0u, 0u);
-            *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 64 + 16 * I + i, 16 * J + j)) =
-                make_uint2(0u, 0u);
+          // the items' TMEM loads in one round trip (an item without data reads its quarter's
+          // first chunk, unused)
+          int blk[3], ch[3];
+          bool has[3];
+          uint32_t v0[16], v1[16], v2[16];
+#pragma unroll
+          for (int it = 0; it < 3; ++it) {
+            has[it] = item_at(it, blk[it], ch[it]);
+            if (!has[it] || ch[it] > blk[it]) { blk[it] = has[it] ? blk[it] : bA; ch[it] = has[it] ? ch[it] : 0; }
           }
+          tmem_ld16(tl + TC_D + dcol(blk[0]) + 16 * (ch[0] <= blk[0] ? ch[0] : 0), v0);
+          tmem_ld16(tl + TC_D + dcol(blk[1]) + 16 * (ch[1] <= blk[1] ? ch[1] : 0), v1);
+          tmem_ld16(tl + TC_D + dcol(blk[2]) + 16 * (ch[2] <= blk[2] ? ch[2] : 0), v2);
+          tmem_wait_ld();
+          if (has[0]) put(blk[0], ch[0], v0);
+          if (has[1]) put(blk[1], ch[1], v1);
+          if (has[2]) put(blk[2], ch[2], v2);
+        }
+        // warps 4, 8, 12 and 13 extract nothing: Xsol's upper right 32x32 block is zero
+        if (warp == 4 || warp == 8 || warp == 12 || warp == 13) {
+          const int t = ((warp == 13) ? 3 : (warp >> 2) - 1) * 32 + lane;  // 0..127
+          const int row = t >> 2, cq = 32 + 8 * (t & 3);
+          *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, row, cq)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, 64 + row, cq)) = make_uint4(0, 0, 0, 0);
         }
       }
-      // R1 (warps 0 and 1, while the others finish the extraction): P_I = (I + T_II)^-1; lane
-      // (I, c) computes column c by forward substitution over the rows of block I
+      // X_AA (warp 0) and X_BB (warp 1), each from its two 16x16 diagonal blocks: half-warp h
+      // computes P_h = (I + T_hh)^-1 (lane c: column c, rows by forward substitution), then the
+      // warp forms the block below the diagonal, X_10 = -P_1 (T_10 P_0)
+      float* Ws = reinterpret_cast<float*>(sm + SM_AOP + 16384 + 32 * YP * 4);  // 2 x [16][20]
       if (warp < 2) {
-        named_bar_sync(1, 64);  // both warps' diagonal blocks of T are in Ts
-        const int I = 2 * warp + (lane >> 4), c = lane & 15, base = 16 * I;
-        float x[16];
-        x[0] = (c == 0) ? 1.f : 0.f;
+        __syncwarp();  // this warp's rows of T are in Ts
+        const int h = lane >> 4, c = lane & 15, base = 32 * warp + 16 * h;
+        {
+          float x[16];
+          x[0] = (c == 0) ? 1.f : 0.f;
 #pragma unroll
-        for (int r = 1; r < 16; ++r) {
-          const float* trow = Ts + (base + r) * TP + base;
-          float a0 = 0.f, a1 = 0.f;
+          for (int rr = 1; rr < 16; ++rr) {
+            const float* trow = Ts + (base + rr) * TP + base;
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-          for (int s0 = 0; s0 < r; s0 += 4) {
-            const float4 t4 = *reinterpret_cast<const float4*>(trow + s0);
-            if (s0 + 0 < r) a0 = fmaf(t4.x, x[s0 + 0], a0);
-            if (s0 + 1 < r) a1 = fmaf(t4.y, x[s0 + 1], a1);
-            if (s0 + 2 < r) a0 = fmaf(t4.z, x[s0 + 2], a0);
-            if (s0 + 3 < r) a1 = fmaf(t4.w, x[s0 + 3], a1);
+            for (int s0 = 0; s0 < rr; s0 += 4) {
+              const float4 t4 = *reinterpret_cast<const float4*>(trow + s0);
+              if (s0 + 0 < rr) a0 = fmaf(t4.x, x[s0], a0);
+              if (s0 + 1 < rr) a1 = fmaf(t4.y, x[s0 + 1], a1);
+              if (s0 + 2 < rr) a0 = fmaf(t4.z, x[s0 + 2], a0);
+              if (s0 + 3 < rr) a1 = fmaf(t4.w, x[s0 + 3], a1);
+            }
+            x[rr] = (rr == c) ? 1.f : -(a0 + a1);
           }
-          x[r] = (r == c) ? 1.f : -(a0 + a1);
-        }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Xs[(base + r) * TP + base + c] = x[r];
+          for (int rr = 0; rr < 16; ++rr) Xs[(base + rr) * TP + base + c] = x[rr];
+        }
+        __syncwarp();
+        // 16x16x16 products by the warp: lane = (row i, column half jh), 8 columns each
+        const int b0 = 32 * warp, i = lane & 15, jh = 8 * (lane >> 4);
+        auto prod16 = [&](const float* Lrow, const float* R, int ldr, float2 (&acc)[4]) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int k0 = 0; k0 < 16; k0 += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(Lrow + k0);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const float4 ra = *reinterpret_cast<const float4*>(R + (k0 + kk) * ldr + jh);
+              const float4 rb = *reinterpret_cast<const float4*>(R + (k0 + kk) * ldr + jh + 4);
+              const float2 l2 = make_float2(lv[kk], lv[kk]);
+              acc[0] = __ffma2_rn(l2, make_float2(ra.x, ra.y), acc[0]);
+              acc[1] = __ffma2_rn(l2, make_float2(ra.z, ra.w), acc[1]);
+              acc[2] = __ffma2_rn(l2, make_float2(rb.x, rb.y), acc[2]);
+              acc[3] = __ffma2_rn(l2, make_float2(rb.z, rb.w), acc[3]);
+            }
+          }
+        };
+        float2 acc[4];
+        float* W = Ws + warp * 16 * 20;
+        prod16(Ts + (b0 + 16 + i) * TP + b0, Xs + b0 * TP + b0, TP, acc);  // T_10 P_0
+        *reinterpret_cast<float4*>(W + i * 20 + jh) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+        *reinterpret_cast<float4*>(W + i * 20 + jh + 4) = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
+        __syncwarp();
+        prod16(Xs + (b0 + 16 + i) * TP + b0 + 16, W, 20, acc);  // P_1 (T_10 P_0)
+        float* xo = Xs + (b0 + 16 + i) * TP + b0 + jh;
+        *reinterpret_cast<float4*>(xo) = make_float4(-acc[0].x, -acc[0].y, -acc[1].x, -acc[1].y);
+        *reinterpret_cast<float4*>(xo + 4) = make_float4(-acc[2].x, -acc[2].y, -acc[3].x, -acc[3].y);
+        // (the block above the diagonal, rows 0-15 x columns 16-31, is zero)
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(Xs + (b0 + i) * TP + b0 + 16 + jh) = z4;
+        *reinterpret_cast<float4*>(Xs + (b0 + i) * TP + b0 + 16 + jh + 4) = z4;
       }
       __syncthreads();
       KDA_TS(13);
-      // R2 .. R5 on warps 0-7, one product per warp and round (barriers among those warps only);
-      // warps 8-15 write the diagonal blocks' Xsol meanwhile
+      // Xsol row `row`, columns c0 .. c0 + 3 from x[4] (bf16 hi in rows 0-63, lo in 64-127)
+      auto put_xsol4 = [&](int row, int c0, float x0, float x1, float x2, float x3) {
+        const float4 b4 = *reinterpret_cast<const float4*>(beta_s + c0);
+        const float f0 = x0 * b4.x, f1 = x1 * b4.y, f2 = x2 * b4.z, f3 = x3 * b4.w;
+        const uint2 hi = pack4(f0, f1, f2, f3);
+        const uint2 lo = make_uint2(split_lo(f0, f1, hi.x), split_lo(f2, f3, hi.y));
+        *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, row, c0)) = hi;
+        *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 64 + row, c0)) = lo;
+      };
       if (warp < 8) {
-#pragma unroll 1
-        for (int rd = 0; rd < 4; ++rd) {
-          const SolveOp op = kSolveOps[rd][warp];
-          if (op.sg != 0) {
-            float* F = reinterpret_cast<float*>(sm);
-            bprod(F + op.l, op.ldl, F + op.r, op.ldr, op.c ? F + op.c : nullptr, op.ldc,
-                  (float)op.sg, F + op.o, op.ldo, op.xi, op.xj);
+        // acc = L_i R[:, c0 .. c0+3] over k < 32: row i of L from Lrow, R rows warp-uniform
+        const int i = lane, c0 = 4 * warp;
+        auto prod = [&](const float* Lrow, const float* R, int ldr, float2 (&acc)[2]) {
+          acc[0] = acc[1] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int k0 = 0; k0 < 32; k0 += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(Lrow + k0);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const float4 ra = *reinterpret_cast<const float4*>(R + (k0 + kk) * ldr + c0);
+              const float2 l2 = make_float2(lv[kk], lv[kk]);
+              acc[0] = __ffma2_rn(l2, make_float2(ra.x, ra.y), acc[0]);
+              acc[1] = __ffma2_rn(l2, make_float2(ra.z, ra.w), acc[1]);
+            }
           }
-          if (rd == 0) KDA_TS(22);
-          if (rd < 3) named_bar_sync(2, 256);
-          if (rd == 0) KDA_TS(14);
-          if (rd == 1) KDA_TS(15);
-        }
+        };
+        float2 acc[2];
+        prod(Ts + (32 + i) * TP, Xs, TP, acc);  // Y = T_BA X_AA
+        *reinterpret_cast<float4*>(Ys + i * YP + c0) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+        named_bar_sync(2, 256);
+        KDA_TS(14);
+        prod(Xs + (32 + i) * TP + 32, Ys, YP, acc);  // X_BA = -X_BB Y
+        put_xsol4(32 + i, c0, -acc[0].x, -acc[0].y, -acc[1].x, -acc[1].y);
+        KDA_TS(15);
       } else {
-        const int t = tid - 256, I = t >> 6, i = (t >> 2) & 15, j = 4 * (t & 3);
-        const float4 x4 = *reinterpret_cast<const float4*>(XB(I, I) + i * TP + j);
-        put_xsol(I, I, i, j, x4.x, x4.y, x4.z, x4.w);
+        // the diagonal blocks' Xsol: 2 blocks x 32 rows x 4 column octets, one item a thread
+        const int t = tid - 256;
+        const int base = 32 * (t >> 7), row = (t >> 2) & 31, cq = 8 * (t & 3);
+        const float* xr = Xs + (base + row) * TP + base + cq;
+        const float4 xa = *reinterpret_cast<const float4*>(xr);
+        const float4 xb = *reinterpret_cast<const float4*>(xr + 4);
+        put_xsol4(base + row, base + cq, xa.x, xa.y, xa.z, xa.w);
+        put_xsol4(base + row, base + cq + 4, xb.x, xb.y, xb.z, xb.w);
       }
       KDA_TS(16);
       fence_proxy_async_smem();
