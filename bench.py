@@ -698,6 +698,35 @@ def run_cp(args, rank, world):
     return 0
 
 
+def render_table(path: str) -> str:
+    """The per-workload markdown table of a bench JSON line (the last line of `path` that has a
+    per_config list)."""
+    line = None
+    with open(path) as f:
+        for raw in f:
+            raw = raw.strip()
+            if raw.startswith("{") and '"per_config"' in raw:
+                line = json.loads(raw)
+    if line is None:
+        raise SystemExit(f"{path}: no bench line with per_config")
+    rows = ["| workload | schedule | ms median (p10-p90), 50 calls | token-heads/s | of HBM peak "
+            "| oracle recurrent / chunked, token-heads/s (threads) |",
+            "|---|---|---|---|---|---|"]
+    for r in line["per_config"]:
+        o = r.get("oracle") or {}
+        rec, chk = o.get("recurrent"), o.get("chunked")
+        ora = (f"{rec['value']:.3g} / {chk['value']:.3g} ({rec['cores']})" if rec and chk else "-")
+        rows.append(f"| {r['workload']} | {r['schedule']} | {r['ms_median']:.4f} "
+                    f"({r['ms_p10']:.4f}-{r['ms_p90']:.4f}) | {r['value']:.3g} | "
+                    f"{100 * r['roofline']['frac']:.1f} % | {ora} |")
+    clk = line.get("clocks") or {}
+    rows.append("")
+    rows.append(f"SM clock {clk.get('sm_mhz')} MHz (max {clk.get('sm_max_mhz')}), throttle reasons "
+                f"{clk.get('reasons')}; peak {line['roofline']['peak']} GB/s "
+                f"({line['roofline'].get('peak_source')}).")
+    return "\n".join(rows)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -728,7 +757,12 @@ def main():
     ap.add_argument("--segment-chunks", type=int, default=-1,
                     help="schedule: -1 the planner's choice, 0 whole units, n > 0 segments of n "
                          "chunks (chunk-parallel scan)")
+    ap.add_argument("--table", metavar="BENCH_JSON",
+                    help="print the per-workload markdown table of a saved bench line and exit")
     args = ap.parse_args()
+    if args.table:
+        print(render_table(args.table))
+        return 0
     args.warmup = max(args.warmup, 3)
     args.per_config_calls = max(args.per_config_calls, 50)
     rank = _env_int("RANK", 0)

@@ -6,8 +6,9 @@ Compiles every ``csrc/*.cu`` and ``csrc/*.cpp`` to objects under ``_build/`` (in
 and links ``chunked_kda_prefill_b200/libkda.so`` with the CUDA runtime linked statically, so
 the library loads on a machine without a GPU (its host entry points work there).
 
-``--define`` builds a variant instead (for example ``KDA_SOLVE_L1=1``, a first-level solve
-variant of the ablation): objects under ``_build_<tag>/`` and ``libkda_<tag>.so``, where
+``--define`` builds a variant instead (for example ``KDA_STATE_LO=0``, the state operand without
+its bf16 remainder, or ``KDA_PHASE_TIMING=1``, per-phase clock stamps for
+``kda_forward_debug``): objects under ``_build_<tag>/`` and ``libkda_<tag>.so``, where
 ``<tag>`` joins the definitions; load it with ``KDA_LIB=<path>``.
 """
 from __future__ import annotations
