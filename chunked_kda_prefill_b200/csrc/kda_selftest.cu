@@ -28,6 +28,8 @@ enum : int {
   ST_TF32_SS = 6,  // kind::tf32, A K-major fp32, B K-major fp32 (shared memory)
   ST_TF32_TS = 7,  // kind::tf32, A fp32 from TMEM, B K-major fp32
   ST_TIMEOUT = 8,  // bounded wait on a barrier that nothing arrives on: must give up and report
+  ST_M64 = 9,      // one M=64 MMA (A K-major [64][K], B K-major [N][K]); D = all 128 lanes x 2N
+                   // columns of TMEM as they are, to map where an M=64 accumulator's rows land
 };
 
 constexpr uint32_t kWaitLimit = 1u << 24;
@@ -112,6 +114,40 @@ __global__ void __launch_bounds__(128, 1)
       tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + c0, r);
       tmem_wait_ld();
       for (int c = 0; c < 16; ++c) D[tid * N + c0 + c] = __uint_as_float(r[c]);
+    }
+  } else if (variant == ST_M64) {
+    for (int e = tid; e < 64 * K; e += 128) {
+      const int m = e / K, k = e % K;
+      *reinterpret_cast<__nv_bfloat16*>(sA + sw128_offset(64, m, k)) = A[e];
+    }
+    for (int e = tid; e < N * K; e += 128) {
+      const int n = e / K, k = e % K;
+      *reinterpret_cast<__nv_bfloat16*>(sB + sw128_offset(N, n, k)) = B[e];
+    }
+    // zero the TMEM columns read back below, so untouched cells read as 0
+    for (int c0 = 0; c0 < 2 * N; c0 += 16)
+      tmem_st16_zero(tbase + ((uint32_t)(warp * 32) << 16) + c0);
+    tmem_wait_st();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16(64, N, 0u, 0u);
+      for (int kk = 0; kk < K / 16; ++kk) {
+        const uint64_t ad = smem_desc(smem_u32(sA) + (kk / 4) * (64 * 128) + (kk % 4) * 32, 16, 1024);
+        const uint64_t bd = smem_desc(smem_u32(sB) + (kk / 4) * (N * 128) + (kk % 4) * 32, 16, 1024);
+        mma_ss(tbase, ad, bd, idesc, kk > 0);
+      }
+      mma_commit(bar_a);
+    }
+    if (!mbar_wait_bounded(bar_a, 0, kWaitLimit) && tid == 0) atomicExch(err, 2);
+    tc_fence_after();
+    for (int c0 = 0; c0 < 2 * N; c0 += 16) {
+      uint32_t r[16];
+      tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + c0, r);
+      tmem_wait_ld();
+      for (int c = 0; c < 16; ++c) D[tid * (2 * N) + c0 + c] = __uint_as_float(r[c]);
     }
   } else if (variant == ST_TMA) {
     if (tid == 0) {
@@ -218,7 +254,9 @@ extern "C" __attribute__((visibility("default"))) int kda_selftest(
     int variant, const void* A, const void* B, float* D, int N, int K, void* raw,
     const void* tma_src, int tma_rows, int row0, int* err_dev, void* stream) {
   using namespace kda;
-  if (variant < 0 || variant > ST_TIMEOUT) return 1;
+  if (variant < 0 || variant > ST_M64) return 1;
+  if (variant == ST_M64 && (!A || !B || !D || N < 16 || N > 128 || N % 16 != 0 || (K != 64 && K != 128)))
+    return 1;
   if (variant != ST_TMA && variant != ST_TIMEOUT && (!A || !B || !D || N < 16 || N > 128 || N % 16 != 0)) return 1;
   if (variant != ST_TMA && variant < ST_TF32_SS && K != 64 && K != 128) return 1;
   if ((variant == ST_TF32_SS || variant == ST_TF32_TS) && K != 32 && K != 64) return 1;

@@ -149,3 +149,37 @@ def test_ex2_accuracy(cuda_ok):
     # results below the smallest normal float are flushed to zero (ftz)
     assert np.all(y[xs <= -127.0] <= 2.0 ** -126)
     print(f"ex2.approx.ftz.f32: max relative error {rel.max():.3e} = 2^{np.log2(rel.max()):.2f}")
+
+
+def test_m64_accumulator_layout(cuda_ok):
+    """Where the rows and columns of an M=64 tcgen05 accumulator land in TMEM (cta_group::1,
+    kind::f16).  A = I (64 x 64), so D[m][n] = B[n][m]: one run with B[n][k] = k + 1 marks every
+    cell with its row, one with B[n][k] = n + 1 with its column.  Every (row, column) must land
+    in exactly one (lane, TMEM column) of the 128 lanes x 128 columns read back."""
+    f = _lib()
+    N, K = 64, 64
+    A = torch.eye(64, K).to(torch.bfloat16).cuda()
+    kk = torch.arange(K, dtype=torch.float32)
+    nn = torch.arange(N, dtype=torch.float32)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    s = torch.cuda.current_stream()
+    raw = []
+    for B in ((kk[None, :] + 1).expand(N, K), (nn[:, None] + 1).expand(N, K)):
+        D = torch.full((128, 2 * N), -1.0, dtype=torch.float32, device="cuda")
+        Bd = B.contiguous().to(torch.bfloat16).cuda()
+        assert f(9, A.data_ptr(), Bd.data_ptr(), D.data_ptr(), N, K, None, None, 0, 0,
+                 err.data_ptr(), s.cuda_stream) == 0
+        raw.append(D.cpu().numpy())
+    rows, cols = raw
+    cells = {}
+    for lane in range(128):
+        for col in range(2 * N):
+            if rows[lane, col] > 0:
+                m, n = int(rows[lane, col]) - 1, int(cols[lane, col]) - 1
+                assert (m, n) not in cells, f"row {m} column {n} found twice"
+                cells[(m, n)] = (lane, col)
+    assert len(cells) == 64 * N, f"{len(cells)} of {64 * N} cells found"
+    # measured on B200: row m in lane (m % 16) + 32 (m / 16), i.e. the first 16 lanes of each
+    # warp's lane quarter; column n in TMEM column n
+    for (m, n), (lane, col) in cells.items():
+        assert lane == (m % 16) + 32 * (m // 16) and col == n, (m, n, lane, col)
