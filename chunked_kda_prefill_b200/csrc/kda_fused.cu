@@ -12,8 +12,9 @@
 //   2 MMA  D_I = Aop B^(I)^T, I = 0..3 (M=128, N=160 for all four blocks, K=128): rows 0-63 give
 //     T = stril(diag(beta) K~ K-^T), rows 64-127 give Aqk = tril(Q~ K-^T); meanwhile K^ lo is
 //     stored and the state left by the previous chunk becomes the bf16 hi/lo state operand
-//   3 solve (CUDA cores, fp32): X = (I+T)^-1 by 32x32 blocks (diagonal inverses by forward
-//     substitution in registers, then the off-diagonal block by two block products);
+//   3 solve (fp32): X = (I+T)^-1 by 32x32 blocks (diagonal inverses by forward substitution in
+//     registers, then the off-diagonal block by two 32x32x32 products on warp-level bf16 MMAs
+//     with a three-term hi/lo split);
 //     Xsol = X diag(beta) -> bf16 hi and lo parts stacked as one 128-row operand
 //   4 MMA  W^T = K~^T [Xsol_hi; Xsol_lo]^T and U^T = V^T [Xsol_hi; Xsol_lo]^T (one N=128 chain
 //          each, hi and lo parts side by side); S <- S Diag(2^G_last)
@@ -99,7 +100,8 @@ constexpr uint32_t SM_BAR = 230144;   // raw_full[2], mma, mma_u (the U MMAs of 
 constexpr uint32_t SM_TSLOT = 230176;
 constexpr uint32_t SM_FLAG = 230180;
 constexpr uint32_t SM_PROD = 230184;  // the TMA producer's state (thread 0 only), 120 bytes
-constexpr uint32_t SM_END = 230304;
+constexpr uint32_t SM_BAR_P1 = 230304;  // one arrival per warp once its phase-1 loads are done
+constexpr uint32_t SM_END = 230312;
 constexpr size_t kFusedSmemBytes = SM_END + 1024;
 
 // per-(block, column) constants of the operand factorisation, indices into SM_CST
@@ -155,6 +157,19 @@ __device__ __forceinline__ uint32_t split_lo(float a, float b, uint32_t hi) {
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
+}
+
+// d += a b for one 16x8x16 tile on the warp-level tensor-core path (bf16 inputs, fp32 d), with the
+// PTX fragment layouts, g = lane / 4 and t = lane % 4: a = A(g, 2t..2t+1), A(g+8, 2t..), A(g, 2t+8..),
+// A(g+8, 2t+8..) (bf16 pairs, first element in the low half); b = B(2t..2t+1, g), B(2t+8..2t+9, g);
+// d = D(g, 2t), D(g, 2t+1), D(g+8, 2t), D(g+8, 2t+1).
+__device__ __forceinline__ void mma_bf16_m16n8k16(float (&d)[4], const uint32_t (&a)[4],
+                                                  const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 struct Maps {
@@ -313,7 +328,7 @@ struct Producer {
   int ld_valid, ld_c, ld_slot;
   LoadRec ld_rec;
 };
-static_assert(sizeof(Producer) <= SM_END - SM_PROD, "producer state overflows its region");
+static_assert(sizeof(Producer) <= SM_BAR_P1 - SM_PROD, "producer state overflows its region");
 
 // Tensor coordinates of chunk c of unit `ur` for the q/k maps (qc) and the v/g/out maps (vc).
 __device__ __forceinline__ void chunk_coords(const Params& p, const LoadRec& ur, int c, int& qc1,
@@ -387,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(sbase + SM_BAR + 8, 8);
     mbar_init(bar_mma, 1);
     mbar_init(bar_mma_u, 1);
+    mbar_init(sbase + SM_BAR_P1, kThreads / 32);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -452,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t gidx = 0;       // chunks consumed by this CTA
   uint32_t mma_phase = 0;    // parity of the next MMA-barrier completion
   uint32_t mma_u_phase = 0;  // and of the phase-4 U MMAs' barrier
+  uint32_t p1_phase = 0;     // and of the phase-1 load barrier
   bool aborted = false;
 
   auto fail = [&]() {
@@ -666,7 +683,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           k4[v][3] = x.w;
         }
       }
-      __syncthreads();
+      // G (in the Aop region) and wtot / the constants (in the B-tile region) are overwritten
+      // below: each warp reports its loads done, and every thread waits for all sixteen reports
+      // only before its first store into those regions
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sbase + SM_BAR_P1);
       KDA_TS(12);
       uint2 khlo[4];  // K^ lo parts of this thread's rows, stored under the intra MMAs
       {
@@ -711,7 +732,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float y = (u4 ? x2[1] : x2[0]) + __shfl_xor_sync(0xffffffffu, u4 ? x2[0] : x2[1], 4);
           y += __shfl_xor_sync(0xffffffffu, y, 2);
           y += __shfl_xor_sync(0xffffffffu, y, 1);
-          // lane l holds the total of value (l >> 2) & 7: index k + 2 (u8) + 4 (u16) of rq (0-3), rk (4-7)
+          // lane l holds the total of value (l >> 2) & 7: index k + 2 (u8) + 4 (u16) of rq (0-3),
+          // rk (4-7); it turns its total into the row's factor (q rows carry the scale), and the
+          // eight factors are broadcast
+          y = rsqrtf(y + 1e-6f) * (u16 ? 1.0f : p.scale);
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
             rqv[m] = __shfl_sync(0xffffffffu, y, 4 * (m & 1) + 8 * (m >> 1));
@@ -726,8 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const int r = r0 + i;
           const bool valid = r < n;
-          const float rq = rsqrtf(rqv[i] + 1e-6f) * p.scale;
-          const float rk = rsqrtf(rkv[i] + 1e-6f);
+          const float rq = rqv[i], rk = rkv[i];
           const float2 rq2 = f2(rq, rq), rk2 = f2(rk, rk);
           uint32_t pa[2], pq[2], pqt[2], pkh[2], pkt[2], pb0[2], pb1[2], pb2[2], pb3[2], pkl[2];
 #pragma unroll
@@ -761,6 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pb3[h] = pack_bf16(b3.x, b3.y);
           }
           khlo[i] = make_uint2(pkl[0], pkl[1]);
+          if (i == 0 && !mbar_wait_bounded(sbase + SM_BAR_P1, p1_phase, kWaitLimit)) fail();
           uint8_t* aop = sm + SM_AOP + colhalf * 16384u + io[i];
           uint8_t* bst = sm + SM_BT + colhalf * (BT_ROWS * 128u) + io[i];
           *reinterpret_cast<uint2*>(aop) = make_uint2(pa[0], pa[1]);
@@ -779,6 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint2*>(sq + OFF_V + colhalf * QGV_ATOM + io[i]) = make_uint2(0, 0);
         }
       }
+      p1_phase ^= 1u;
       if (st_thread) tma_store_wait_read();  // the previous out tile (in the K^ lo region) was read
       fence_proxy_async_smem();
       tc_fence_before();
@@ -813,13 +838,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the intra MMAs.  16 state columns at a time; warp 0 issues the MMAs, so warps 8 and
         // 12 (its TMEM lanes) take its columns.  (D = 64: columns past D stay out of every
         // product, phase 5 skipping their K steps.)
-        auto conv16 = [&](int c16) {
-          uint32_t v[16], hi[8];
+        auto conv16_of = [&](int c16, const uint32_t (&v)[16]) {
+          uint32_t hi[8];
 #if KDA_STATE_LO
           uint32_t lo[8];
 #endif
-          tmem_ld16(tl + TC_S + c16, v);
-          tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float a0 = __uint_as_float(v[2 * e]), a1 = __uint_as_float(v[2 * e + 1]);
@@ -833,9 +856,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st8(tl + TC_SLO + c16 / 2, lo);
 #endif
         };
+        auto conv16 = [&](int c16) {
+          uint32_t v[16];
+          tmem_ld16(tl + TC_S + c16, v);
+          tmem_wait_ld();
+          conv16_of(c16, v);
+        };
         if (warp != 0 && wg * 32 < DIM) {
-          conv16(wg * 32);
-          conv16(wg * 32 + 16);
+          uint32_t va[16], vb[16];
+          tmem_ld16(tl + TC_S + wg * 32, va);
+          tmem_ld16(tl + TC_S + wg * 32 + 16, vb);
+          tmem_wait_ld();
+          conv16_of(wg * 32, va);
+          conv16_of(wg * 32 + 16, vb);
         }
         if (warp == 8) conv16(0);
         if (warp == 12) conv16(16);
@@ -851,8 +884,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       //     rows of T: two 16x16 diagonal inverses by column forward substitution (a half-warp
       //     each, lane c computing column c in registers) and the block below them,
       //     X_10 = -P_1 (T_10 P_0), by two 16x16x16 products;
-      //   X_BA = -X_BB (T_BA X_AA), two 32x32x32 products on warps 0-7 (lane i owns row i, warp w
-      //     columns 4w .. 4w+3; the right-hand operand is read warp-uniformly, a broadcast);
+      //   X_BA = -X_BB (T_BA X_AA), two 32x32x32 products on warps 0-7 (one 16x8 output tile a
+      //     warp, on the warp-level tensor-core path);
       // Xsol = X diag(beta) goes out in bf16 hi and lo parts, the diagonal blocks by warps 8-15
       // while the products run.
       constexpr int TP = 68;                              // row pitch of T and X (floats)
@@ -949,6 +982,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // computes P_h = (I + T_hh)^-1 (lane c: column c, rows by forward substitution), then the
       // warp forms the block below the diagonal, X_10 = -P_1 (T_10 P_0)
       float* Ws = reinterpret_cast<float*>(sm + SM_AOP + 16384 + 32 * YP * 4);  // 2 x [16][20]
+      KDA_TS(19);
       if (warp < 2) {
         __syncwarp();  // this warp's rows of T are in Ts
         const int h = lane >> 4, c = lane & 15, base = 32 * warp + 16 * h;
@@ -973,6 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int rr = 0; rr < 16; ++rr) Xs[(base + rr) * TP + base + c] = x[rr];
         }
         __syncwarp();
+        KDA_TS(20);
         // 16x16x16 products by the warp: lane = (row i, column half jh), 8 columns each
         const int b0 = 32 * warp, i = lane & 15, jh = 8 * (lane >> 4);
         auto prod16 = [&](const float* Lrow, const float* R, int ldr, float2 (&acc)[4]) {
@@ -1000,6 +1035,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<float4*>(W + i * 20 + jh) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
         *reinterpret_cast<float4*>(W + i * 20 + jh + 4) = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
         __syncwarp();
+        KDA_TS(21);
         prod16(Xs + (b0 + 16 + i) * TP + b0 + 16, W, 20, acc);  // P_1 (T_10 P_0)
         float* xo = Xs + (b0 + 16 + i) * TP + b0 + jh;
         *reinterpret_cast<float4*>(xo) = make_float4(-acc[0].x, -acc[0].y, -acc[1].x, -acc[1].y);
@@ -1008,6 +1044,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<float4*>(Xs + (b0 + i) * TP + b0 + 16 + jh) = z4;
         *reinterpret_cast<float4*>(Xs + (b0 + i) * TP + b0 + 16 + jh + 4) = z4;
+        KDA_TS(22);
       }
       __syncthreads();
       KDA_TS(13);
@@ -1021,30 +1058,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint2*>(sm + SM_XSOL + sw128_offset(128, 64 + row, c0)) = lo;
       };
       if (warp < 8) {
-        // acc = L_i R[:, c0 .. c0+3] over k < 32: row i of L from Lrow, R rows warp-uniform
-        const int i = lane, c0 = 4 * warp;
-        auto prod = [&](const float* Lrow, const float* R, int ldr, float2 (&acc)[2]) {
-          acc[0] = acc[1] = make_float2(0.f, 0.f);
+        // d = L R for the warp's 16x8 tile (rows 16 mt.., columns 8 nt..) of a 32x32x32 product,
+        // on the warp-level tensor-core path (mma.sync m16n8k16, bf16).  Each operand is split
+        // into a bf16 high part and a bf16 remainder and multiplied as lo*hi + hi*lo + hi*hi
+        // (about 16 significant bits, as the Xsol operand these blocks become; fp32
+        // accumulation).  This reads a small fraction of the shared-memory wavefronts of the
+        // FFMA form, where every lane needs a whole row of L and a broadcast of R, and issues
+        // half the instructions of the tf32 m16n8k8 form.
+        const int mt = warp >> 2, nt = warp & 3, g = lane >> 2, t = lane & 3;
+        auto tprod = [&](const float* L, int ldl, const float* R, int ldr, float (&d)[4]) {
+          d[0] = d[1] = d[2] = d[3] = 0.f;
+          float2 av[2][4];
+          float bv[2][4];
 #pragma unroll
-          for (int k0 = 0; k0 < 32; k0 += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(Lrow + k0);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          for (int ks = 0; ks < 2; ++ks) {
+            const int k0 = 16 * ks + 2 * t;
+            av[ks][0] = *reinterpret_cast<const float2*>(L + g * ldl + k0);
+            av[ks][1] = *reinterpret_cast<const float2*>(L + (g + 8) * ldl + k0);
+            av[ks][2] = *reinterpret_cast<const float2*>(L + g * ldl + k0 + 8);
+            av[ks][3] = *reinterpret_cast<const float2*>(L + (g + 8) * ldl + k0 + 8);
+            bv[ks][0] = R[k0 * ldr + g];
+            bv[ks][1] = R[(k0 + 1) * ldr + g];
+            bv[ks][2] = R[(k0 + 8) * ldr + g];
+            bv[ks][3] = R[(k0 + 9) * ldr + g];
+          }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const float4 ra = *reinterpret_cast<const float4*>(R + (k0 + kk) * ldr + c0);
-              const float2 l2 = make_float2(lv[kk], lv[kk]);
-              acc[0] = __ffma2_rn(l2, make_float2(ra.x, ra.y), acc[0]);
-              acc[1] = __ffma2_rn(l2, make_float2(ra.z, ra.w), acc[1]);
+          for (int ks = 0; ks < 2; ++ks) {
+            uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              ah[e] = pack_bf16(av[ks][e].x, av[ks][e].y);
+              al[e] = split_lo(av[ks][e].x, av[ks][e].y, ah[e]);
             }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              bh[e] = pack_bf16(bv[ks][2 * e], bv[ks][2 * e + 1]);
+              bl[e] = split_lo(bv[ks][2 * e], bv[ks][2 * e + 1], bh[e]);
+            }
+            mma_bf16_m16n8k16(d, al, bh);
+            mma_bf16_m16n8k16(d, ah, bl);
+            mma_bf16_m16n8k16(d, ah, bh);
           }
         };
-        float2 acc[2];
-        prod(Ts + (32 + i) * TP, Xs, TP, acc);  // Y = T_BA X_AA
-        *reinterpret_cast<float4*>(Ys + i * YP + c0) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+        float d[4];
+        tprod(Ts + (32 + 16 * mt) * TP, TP, Xs + 8 * nt, TP, d);  // Y = T_BA X_AA
+        const int yr = 16 * mt + g, yc = 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(Ys + yr * YP + yc) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(Ys + (yr + 8) * YP + yc) = make_float2(d[2], d[3]);
         named_bar_sync(2, 256);
         KDA_TS(14);
-        prod(Xs + (32 + i) * TP + 32, Ys, YP, acc);  // X_BA = -X_BB Y
-        put_xsol4(32 + i, c0, -acc[0].x, -acc[0].y, -acc[1].x, -acc[1].y);
+        tprod(Xs + (32 + 16 * mt) * TP + 32, TP, Ys + 8 * nt, YP, d);  // X_BA = -X_BB Y
+        // Xsol rows 32 + yr and 40 + yr, columns yc and yc + 1 (bf16 hi in rows 0-63, lo in 64-127)
+        const float2 b2 = *reinterpret_cast<const float2*>(beta_s + yc);
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const float f0 = -d[2 * hr] * b2.x, f1 = -d[2 * hr + 1] * b2.y;
+          const uint32_t hi = pack_bf16(f0, f1);
+          const int row = 32 + yr + 8 * hr;
+          *reinterpret_cast<uint32_t*>(sm + SM_XSOL + sw128_offset(128, row, yc)) = hi;
+          *reinterpret_cast<uint32_t*>(sm + SM_XSOL + sw128_offset(128, 64 + row, yc)) =
+              split_lo(f0, f1, hi);
+        }
         KDA_TS(15);
       } else {
         // the diagonal blocks' Xsol: 2 blocks x 32 rows x 4 column octets, one item a thread
