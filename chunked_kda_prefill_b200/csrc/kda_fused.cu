@@ -898,8 +898,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // TMEM lane quarter q4 = warp & 3 holds rows 32 (q4 & 1) .. +31 of k (q4 < 2) or q (q4 >= 2),
         // i.e. row blocks bA = 2 (q4 & 1) and bA + 1.  Items are (16-row block, 16-column chunk);
         // chunks right of a block's diagonal are zero.  q rows (Aqk): the quarter's 8 items, 2 a
-        // warp.  k rows (T): warp 0 takes T_AA's three chunks (0,0) (1,0) (1,1) and warp 1 T_BB's
-        // (2,2) (3,2) (3,3), so each can start its diagonal inverse at once; warps 5 and 9 take T_BA.
+        // warp.  k rows (T): T_AA's three chunks (0,0) (1,0) (1,1) go to warps 0, 4 and 8, and T_BB's
+        // (2,2) (3,2) (3,3) to warps 1, 5 and 9, one each and first, so that warps 0 and 1 (the
+        // diagonal inverses) wait only for one extraction; T_BA's four chunks go to warps 5, 9 and 13.
         const int q4 = warp & 3;
         const int r = (q4 & 1) * 32 + lane;
         const bool krow = q4 < 2;
@@ -907,14 +908,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bA = 2 * (q4 & 1);
         auto item_at = [&](int it, int& blk, int& ch) -> bool {
           if (krow) {
-            if (wg == 0) {
-              blk = bA + (it > 0 ? 1 : 0);
-              ch = bA + (it == 2 ? 1 : 0);
+            if (it == 0 && wg < 3) {  // the diagonal block pair: (bA,bA) (bA+1,bA) (bA+1,bA+1)
+              blk = bA + (wg > 0 ? 1 : 0);
+              ch = bA + (wg == 2 ? 1 : 0);
               return true;
             }
-            blk = 2 + (it & 1);  // warp 5: (2,0) (3,0); warp 9: (2,1) (3,1)
-            ch = wg - 1;
-            return q4 == 1 && (wg == 1 || wg == 2) && it < 2;
+            // T_BA: warp 5 (2,1); warp 9 (3,1); warp 13 (2,0) (3,0)
+            blk = (wg == 3) ? 2 + it : wg + 1;
+            ch = (wg == 3) ? 0 : 1;
+            return q4 == 1 && wg >= 1 && (wg == 3 || it == 1);
           }
           const int item = 2 * wg + it;
           blk = bA + (item >> 2);
@@ -954,28 +956,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           // the items' TMEM loads in one round trip (an item without data reads its quarter's
           // first chunk, unused)
-          int blk[3], ch[3];
-          bool has[3];
-          uint32_t v0[16], v1[16], v2[16];
+          int blk[2], ch[2];
+          bool has[2];
+          uint32_t v0[16], v1[16];
 #pragma unroll
-          for (int it = 0; it < 3; ++it) {
+          for (int it = 0; it < 2; ++it) {
             has[it] = item_at(it, blk[it], ch[it]);
             if (!has[it] || ch[it] > blk[it]) { blk[it] = has[it] ? blk[it] : bA; ch[it] = has[it] ? ch[it] : 0; }
           }
+          KDA_TS(24);
           tmem_ld16(tl + TC_D + dcol(blk[0]) + 16 * (ch[0] <= blk[0] ? ch[0] : 0), v0);
           tmem_ld16(tl + TC_D + dcol(blk[1]) + 16 * (ch[1] <= blk[1] ? ch[1] : 0), v1);
-          tmem_ld16(tl + TC_D + dcol(blk[2]) + 16 * (ch[2] <= blk[2] ? ch[2] : 0), v2);
           tmem_wait_ld();
+          KDA_TS(23);
           if (has[0]) put(blk[0], ch[0], v0);
+          // the second and third chunk of T_AA / T_BB are in Ts: tell warp 0 / 1
+          if (krow && (wg == 1 || wg == 2)) named_bar_arrive(3 + q4, 96);
           if (has[1]) put(blk[1], ch[1], v1);
-          if (has[2]) put(blk[2], ch[2], v2);
         }
-        // warps 4, 8, 12 and 13 extract nothing: Xsol's upper right 32x32 block is zero
-        if (warp == 4 || warp == 8 || warp == 12 || warp == 13) {
-          const int t = ((warp == 13) ? 3 : (warp >> 2) - 1) * 32 + lane;  // 0..127
-          const int row = t >> 2, cq = 32 + 8 * (t & 3);
-          *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, row, cq)) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, 64 + row, cq)) = make_uint4(0, 0, 0, 0);
+        // warp 12 extracts nothing: Xsol's upper right 32x32 block is zero
+        if (warp == 12) {
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int t = 32 * k4 + lane;  // 0..127
+            const int row = t >> 2, cq = 32 + 8 * (t & 3);
+            *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, row, cq)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sm + SM_XSOL + sw128_offset(128, 64 + row, cq)) = make_uint4(0, 0, 0, 0);
+          }
         }
       }
       // X_AA (warp 0) and X_BB (warp 1), each from its two 16x16 diagonal blocks: half-warp h
@@ -984,7 +991,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* Ws = reinterpret_cast<float*>(sm + SM_AOP + 16384 + 32 * YP * 4);  // 2 x [16][20]
       KDA_TS(19);
       if (warp < 2) {
-        __syncwarp();  // this warp's rows of T are in Ts
+        named_bar_sync(3 + warp, 96);  // this warp's rows of T are in Ts (its chunk and warps 4/8's or 5/9's)
         const int h = lane >> 4, c = lane & 15, base = 32 * warp + 16 * h;
         {
           float x[16];
@@ -1278,6 +1285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tbase + TC_O, tbase + TC_SLO + kk * 8, bd, idesc_2, 1);
         }
 #endif
+        KDA_TS(26);
         mma_commit(bar_mma);
       }
       if (c + 1 < it.c_end) {
@@ -1328,6 +1336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tbase + TC_O, tbase + TC_DHI + kk * 8, smem_desc(sbase + SM_AQK + kk * 32, 16, 1024),
                  idesc_o, 1);
         }
+        KDA_TS(25);
         mma_commit(bar_mma);
       }
       if (lane == 0 && warp >= 1 && warp <= 6) issue_planned(warp - 1);  // q/g/v of this slot are free
