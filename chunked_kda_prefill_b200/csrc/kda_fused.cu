@@ -85,8 +85,6 @@ constexpr uint32_t QGV_ATOM = 24576;  // distance between the two column halves 
 constexpr uint32_t K_ATOM = 8192;
 constexpr uint32_t SM_AOP = 131072;   // [128 rows][128] bf16, 2 atoms of 16 KB; after phase 2:
 constexpr uint32_t SM_XSOL = SM_AOP;  //   [Xsol hi ; Xsol lo] 128 rows x 64 cols (16 KB)
-constexpr uint32_t SM_GT = SM_AOP;    //   from phase 5: the next chunk's in-warp gate cumsums,
-                                      //   fp32 [64][128] (read back in its phase 1)
 constexpr uint32_t SM_BT = 163840;    // [B^(0); B^(1); B^(2); B^(3)]: one 160-row tile; the solve
 constexpr uint32_t BT_ROWS = 160;     //   scratch in phase 3; from phase 5 the next chunk's
 constexpr uint32_t SM_WTOT = SM_BT;   //   warp totals / prefixes fp32 [16][128] and
@@ -393,7 +391,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_FLAG);
   float* wtot = reinterpret_cast<float*>(sm + SM_WTOT);
   float* cst = reinterpret_cast<float*>(sm + SM_CST);
-  float* gtile = reinterpret_cast<float*>(sm + SM_GT);
   float* gcs = reinterpret_cast<float*>(sm + SM_GC);
   float* beta_s = reinterpret_cast<float*>(sm + SM_BETA);
 
@@ -549,18 +546,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // The front of phase 1 of chunk cc (ring slot of the gi-th chunk of this CTA): wait for its
-    // tiles; gate activation and the in-thread cumsum of this thread's 4 rows -> the G tile,
-    // warp totals -> wtot; beta.  For every chunk after an item's first it runs under the
-    // previous chunk's phase-5 MMAs (the G tile and wtot regions are free from then on).
+    // tiles; gate activation and the in-thread cumsum of this thread's 4 rows (kept in registers
+    // until that phase 1), warp totals -> wtot; beta.  For every chunk after an item's first it
+    // runs under the previous chunk's phase-5 MMAs (warp 0 after issuing them; the wtot region is
+    // free from then on).
+    float4 gnext[4];  // this thread's rows of the next chunk's in-warp cumsums (front_gate -> phase 1)
     auto front_gate = [&](int cc, uint32_t gi, __nv_bfloat16 blog) {
       const int nn = min(kChunk, L - cc * kChunk);
       const uint8_t* sg_tile = sm + (gi & 1) * SLOT_BYTES + OFF_G;
       if (!mbar_wait_bounded(sbase + SM_BAR + 8u * (gi & 1), (gi >> 1) & 1u, kWaitLimit)) fail();
       // g_act * log2(e) = lb log2(e) / (1 + 2^(-log2(e) e^A_log (g_raw + dt_bias)))
       const float ca = -a_h * kLog2e;
-      // rows 4 grp .. 4 grp + 3; warp 0 issues the MMAs this overlaps, so warp 4 (the same SM
-      // sub-partition) takes its rows as well
-      auto group = [&](int grp) {
+      // this thread's rows 4 warp .. 4 warp + 3 and columns j0 .. j0 + 3 (the phase-1 map), kept in
+      // registers until phase 1; the warp totals go to wtot for the column scan
+      {
+        const int grp = warp;
         float2 G[4][2];  // rows x column pairs (packed fp32x2 arithmetic)
         const float2 ca2 = make_float2(ca, ca), one2 = make_float2(1.f, 1.f);
         const float2 lb2 = make_float2(lbl2, lbl2);
@@ -568,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const int r = 4 * grp + i;
           // (row 4 grp + i has the swizzle of row r0 + i: grp and warp have the same parity)
-          const int off = (int)(colhalf * QGV_ATOM + io[i]) + (grp - warp) * 512;
+          const int off = (int)(colhalf * QGV_ATOM + io[i]);
           const uint2 w = *reinterpret_cast<const uint2*>(sg_tile + off);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -588,16 +588,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             G[i][0] = __fadd2_rn(G[i][0], G[i - 1][0]);
             G[i][1] = __fadd2_rn(G[i][1], G[i - 1][1]);
           }
-          *reinterpret_cast<float4*>(gtile + (4 * grp + i) * kD + j0) =
-              make_float4(G[i][0].x, G[i][0].y, G[i][1].x, G[i][1].y);
+          gnext[i] = make_float4(G[i][0].x, G[i][0].y, G[i][1].x, G[i][1].y);
         }
         *reinterpret_cast<float4*>(wtot + grp * kD + j0) =
             make_float4(G[3][0].x, G[3][0].y, G[3][1].x, G[3][1].y);
-      };
-      // (one call site: warp 4 runs it twice)
-#pragma unroll 1
-      for (int rep = (warp == 4) ? 0 : 1; rep < 2; ++rep)
-        if (warp != 0) group(rep == 0 ? 0 : warp);
+      }
       if (tid >= kChunk && tid < 2 * kChunk)  // (beta: threads 64-127, not warp 0)
         beta_s[tid - kChunk] =
             (tid - kChunk < nn) ? __fdividef(1.0f, 1.0f + __expf(-__bfloat162float(blog))) : 0.0f;
@@ -663,12 +658,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       float G[4][4];
       float k4[CST_N][4];
       {
-        // this thread's rows of G (in-warp cumsum + the warp prefix) and its block's constants,
-        // all read before any thread overwrites the regions they live in
+        // this thread's rows of G (in-warp cumsum + the warp prefix) and its block's constants
         const float4 pre = *reinterpret_cast<const float4*>(wtot + warp * kD + j0);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float4 x = *reinterpret_cast<const float4*>(gtile + (r0 + i) * kD + j0);
+          const float4 x = gnext[i];
           G[i][0] = x.x + pre.x;
           G[i][1] = x.y + pre.y;
           G[i][2] = x.z + pre.z;
@@ -683,9 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           k4[v][3] = x.w;
         }
       }
-      // G (in the Aop region) and wtot / the constants (in the B-tile region) are overwritten
-      // below: each warp reports its loads done, and every thread waits for all sixteen reports
-      // only before its first store into those regions
+      // wtot and the constants (in the B-tile region) are overwritten below by the staircase:
+      // each warp reports its loads done, and every thread waits for all sixteen reports only
+      // before its first store into that region
       __syncwarp();
       if (lane == 0) mbar_arrive(sbase + SM_BAR_P1);
       KDA_TS(12);
