@@ -1,6 +1,7 @@
 // kda_api.cu -- kda_forward / kda_device_status: argument checks, then the kernel launches.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -126,7 +127,8 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   p.seg_chunks = plan_host[PH_SEG_CHUNKS];
   p.states = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWsHeaderBytes);
 
-  if (cudaMemsetAsync(workspace, 0, 4, stream) != cudaSuccess) return KDA_ERR_CUDA;
+  // the status word and the item counter of a dynamically scheduled launch
+  if (cudaMemsetAsync(workspace, 0, 8, stream) != cudaSuccess) return KDA_ERR_CUDA;
   cudaError_t e;
   if (path == PATH_SIMT) {
     e = launch_simt(p, plan_host[PH_TOTAL_CHUNKS], stream);
@@ -146,7 +148,15 @@ kda_status_t forward_impl(int path, const kda_shape_t* shape, const int32_t* pla
   } else if (p.seg_chunks <= 0) {
     p.mode = 0;
     p.n_items = p.n_units;
-    e = launch_fused(p, dbg, stream);
+    // units of different lengths are claimed dynamically, longest first (the plan's order), by
+    // whichever CTA frees up first; equal units keep the fixed stride
+    const int32_t* R = plan_host + kPlanHeader;
+    int lo = INT_MAX, hi = 0;
+    for (int u = 0; u < p.n_units; ++u) {
+      lo = std::min(lo, (int)R[u * kPlanRecord + PR_CHUNKS]);
+      hi = std::max(hi, (int)R[u * kPlanRecord + PR_CHUNKS]);
+    }
+    e = launch_fused(p, dbg, stream, hi > lo);
   } else {
     // segmented schedule: segment summaries, start states, outputs
     const SegCounts sc = seg_counts(plan_host);

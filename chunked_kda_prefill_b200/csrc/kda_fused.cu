@@ -317,14 +317,21 @@ __device__ __forceinline__ LoadRec load_rec(const Params& p, int i) {
 
 // The load schedule, kept in shared memory: the cursor (next (item, chunk) of this CTA's stream,
 // chunks planned so far, the current and next item, read one item ahead so no global load sits
-// on the issue path), written by thread 0 only; and the chunk whose tiles go out during the
-// current chunk, which ten warps read to issue one TMA box each.
+// on the issue path), written by thread 0 only; the chunk whose tiles go out during the current
+// chunk, which ten warps read to issue one TMA box each; and, in the dynamically scheduled
+// instance, the CTA's item sequence.  There a CTA's first item is its blockIdx.x and thread 0
+// claims each later one from the launch's item counter when its loads reach the item before
+// (items go out in plan order, longest first, to whichever CTA frees up first); the consumer
+// loop reads the sequence from a ring of four, as the loads run at most two chunks, so at most
+// three items, ahead of it.  The other instances take every gridDim.x-th item.
 struct Producer {
   int pu, pc;
   uint32_t issued;
   LoadRec cur, next;
   int ld_valid, ld_c, ld_slot;
   LoadRec ld_rec;
+  int next_item, n_seq;
+  int seq[4];
 };
 static_assert(sizeof(Producer) <= SM_BAR_P1 - SM_PROD, "producer state overflows its region");
 
@@ -365,7 +372,9 @@ __device__ __forceinline__ void issue_box(const Params& p, const Maps& m, uint32
 // TMEM accumulator and MMA is 128 channels wide either way.  KIND: KIND_FORWARD (modes 0-2),
 // KIND_SUMMARY (mode 3), or KIND_DEBUG (mode 0 that also dumps every chunk's intermediates to
 // `dbg`; a separate instance, so the dump code takes no registers from the others).
-enum : int { KIND_FORWARD = 0, KIND_SUMMARY = 1, KIND_DEBUG = 2 };
+// KIND_FORWARD_DYN: mode 0 with dynamic item claims, for plans whose units differ in length and
+// outnumber the CTAs.
+enum : int { KIND_FORWARD = 0, KIND_SUMMARY = 1, KIND_DEBUG = 2, KIND_FORWARD_DYN = 3 };
 template <int DIM, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_kernel(const Params p, const __grid_constant__ Maps maps, float* dbg) {
@@ -415,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tl = tbase + wlane;  // this warp's TMEM lane quarter
 
   const int G_stride = gridDim.x;
+  int32_t* const item_counter = reinterpret_cast<int32_t*>(p.ws + 4);  // (dynamic instance)
   // Thread 0 issues every MMA and plans the loads; the TMA boxes are issued by other warps so no
   // thread carries more than one or two.  Per chunk c (ring slot s): during the phase-2 MMAs
   // thread 0 picks chunk c+2 (slot s again); lane 0 of warps 1-6 issue its q/g/v boxes in phase 7
@@ -433,10 +443,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     pr.ld_slot = pr.issued & 1;
     ++pr.issued;
     if (++pr.pc == pr.cur.c_end) {
-      pr.pu += G_stride;
-      pr.cur = pr.next;
-      pr.pc = pr.cur.c_begin;
-      pr.next = load_rec<DIM, KIND == KIND_SUMMARY>(p, pr.pu + G_stride);
+      if constexpr (KIND == KIND_FORWARD_DYN) {
+        pr.pu = pr.next_item;
+        pr.cur = pr.next;
+        pr.pc = pr.cur.c_begin;
+        pr.next_item = (pr.pu < p.n_items) ? (G_stride + atomicAdd(item_counter, 1)) : p.n_items;
+        pr.next = load_rec<DIM, false>(p, pr.next_item);
+        pr.seq[pr.n_seq & 3] = pr.next_item;
+        ++pr.n_seq;
+      } else {
+        pr.pu += G_stride;
+        pr.cur = pr.next;
+        pr.pc = pr.cur.c_begin;
+        pr.next = load_rec<DIM, KIND == KIND_SUMMARY>(p, pr.pu + G_stride);
+      }
     }
   };
   auto issue_planned = [&](int box) {
@@ -449,7 +469,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     prod->issued = 0;
     prod->cur = load_rec<DIM, KIND == KIND_SUMMARY>(p, blockIdx.x);
     prod->pc = prod->cur.c_begin;
-    prod->next = load_rec<DIM, KIND == KIND_SUMMARY>(p, blockIdx.x + G_stride);
+    if constexpr (KIND == KIND_FORWARD_DYN) {
+      prod->next_item = G_stride + atomicAdd(item_counter, 1);
+      prod->next = load_rec<DIM, false>(p, prod->next_item);
+      prod->seq[0] = blockIdx.x;
+      prod->seq[1] = prod->next_item;
+      prod->n_seq = 2;
+    } else {
+      prod->next = load_rec<DIM, KIND == KIND_SUMMARY>(p, blockIdx.x + G_stride);
+    }
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.k);
     tma_prefetch_desc(&maps.v);
@@ -461,6 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     prod->ld_valid = 0;
   }
+  if constexpr (KIND == KIND_FORWARD_DYN) __syncthreads();  // the sequence's first entries
 
   uint32_t gidx = 0;       // chunks consumed by this CTA
   uint32_t mma_phase = 0;    // parity of the next MMA-barrier completion
@@ -491,7 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const uint32_t colhalf = (uint32_t)(j0 >> 6);
 
-  for (int ii = blockIdx.x; ii < p.n_items && !aborted; ii += G_stride) {
+  for (int k_item = 0, ii = blockIdx.x; ii < p.n_items && !aborted;
+       ++k_item, ii = (KIND == KIND_FORWARD_DYN) ? prod->seq[k_item & 3] : ii + G_stride) {
     const Item it = item_of<DIM, KIND == KIND_SUMMARY>(p, ii);
     const int b = it.b, h = it.h, tok0 = it.tok0, L = it.L, coff = it.coff;
     const float a_h = expf(p.A_log[h]);
@@ -1461,7 +1491,7 @@ bool make_map(CUtensorMap* m, const void* base, int layout, int B, int NX, int S
 
 }  // namespace
 
-cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
+cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream, bool dyn_items) {
   static PerDevice setup;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1470,6 +1500,8 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
   e = once_per_device(setup, dev, &num_sms, [](int d, int* sms) {
     const void* fns[] = {(const void*)kda_fused_kernel<kD, KIND_FORWARD>,
                          (const void*)kda_fused_kernel<64, KIND_FORWARD>,
+                         (const void*)kda_fused_kernel<kD, KIND_FORWARD_DYN>,
+                         (const void*)kda_fused_kernel<64, KIND_FORWARD_DYN>,
                          (const void*)kda_fused_kernel<kD, KIND_SUMMARY>,
                          (const void*)kda_fused_kernel<64, KIND_SUMMARY>,
                          (const void*)kda_fused_kernel<kD, KIND_DEBUG>,
@@ -1492,12 +1524,17 @@ cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   if (p.n_items < 1) return cudaSuccess;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
-  const int kind = (p.mode == 3) ? KIND_SUMMARY : dbg ? KIND_DEBUG : KIND_FORWARD;
+  const int kind = (p.mode == 3) ? KIND_SUMMARY
+                   : dbg          ? KIND_DEBUG
+                   : (p.mode == 0 && dyn_items && p.n_items > grid) ? KIND_FORWARD_DYN
+                                                                      : KIND_FORWARD;
   const bool d128 = (p.D == kD);
 #define KDA_LAUNCH_FUSED(DIM_, KIND_) \
   kda_fused_kernel<DIM_, KIND_><<<grid, kThreads, kFusedSmemBytes, stream>>>(p, m, dbg)
   if (kind == KIND_FORWARD) {
     if (d128) KDA_LAUNCH_FUSED(kD, KIND_FORWARD); else KDA_LAUNCH_FUSED(64, KIND_FORWARD);
+  } else if (kind == KIND_FORWARD_DYN) {
+    if (d128) KDA_LAUNCH_FUSED(kD, KIND_FORWARD_DYN); else KDA_LAUNCH_FUSED(64, KIND_FORWARD_DYN);
   } else if (kind == KIND_SUMMARY) {
     if (d128) KDA_LAUNCH_FUSED(kD, KIND_SUMMARY); else KDA_LAUNCH_FUSED(64, KIND_SUMMARY);
   } else {

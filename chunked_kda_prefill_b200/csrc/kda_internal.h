@@ -45,7 +45,7 @@ struct SegCounts {
 SegCounts seg_counts(const int32_t* plan);
 
 // ---- workspace ----
-constexpr size_t kWsHeaderBytes = 256;  // int32 status word at offset 0
+constexpr size_t kWsHeaderBytes = 256;  // int32 status word at offset 0, item counter at 4
 enum DeviceStatus : int32_t { DS_OK = 0, DS_PLAN = 1, DS_TIMEOUT = 2 };
 
 // Per-chunk intermediates of the two-kernel path (fp32):

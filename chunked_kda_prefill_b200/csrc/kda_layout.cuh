@@ -70,7 +70,9 @@ __device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float x[4]) {
 cudaError_t launch_simt(const Params& p, int total_chunks, cudaStream_t stream);
 // The fused tcgen05 path (kda_fused.cu): needs kWsHeaderBytes of workspace.  A non-null `dbg`
 // receives every chunk's intermediates in the two-kernel workspace layout (test aid).
-cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream);
+// dyn_items (mode 0 only): units are claimed dynamically, longest first, from an item counter at
+// workspace offset 4, which must be zero at the launch
+cudaError_t launch_fused(const Params& p, float* dbg, cudaStream_t stream, bool dyn_items = false);
 // The segmented schedule's middle kernel: every unit's segment start states from the segment
 // summaries (S_{s+1} = S_s M_s + R_s, fp32).
 cudaError_t launch_combine(const Params& p, cudaStream_t stream);
